@@ -1,0 +1,19 @@
+"""CPU oracle for the packed-tree SSM scan -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this package.  The CUDA library and its Python binding never import,
+load or call it, and the two share no code.
+
+* ``walk``   -- the plain definition: a fp64 C walk of every node's root path
+               (``stree_oracle.c``), wrapped with ctypes.
+* ``packed`` -- a second fp64 formulation (numpy) of the same outputs through the
+               accumulated transition ``A_tree = L . log A``; used only to
+               cross-check the walk.
+"""
+from .walk import (  # noqa: F401
+    build_oracle,
+    oracle_build_tree,
+    oracle_commit,
+    oracle_max_threads,
+    oracle_tree_scan,
+)
