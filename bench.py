@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the packed-tree SSM scan + commit on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+build the tree masks once, then the fused scan + commit of every layer (y for
+every node, h_new for the accepted path).  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config m2_2p7b]
+    python bench.py --impl reference ...      # the CPU oracle arm
+
+Timing: CUDA events on the launching stream, K steps bracketed by a barrier and
+a synchronize, max over ranks.  Workloads smaller than L2 rotate over enough
+copies of their buffers that each step reads data that is not L2-resident.
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling); the path has
+no exchange step, so no collective touches the data.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tree-scan nodes/sec and achieved HBM GB/s (% of roofline), 1×B200"
+UNIT = "nodes/s"
+DEFAULT_CONFIG = "m2_2p7b"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample budget")
+    return ap.parse_args()
+
+
+def default_steps(name):
+    return {"tiny": 200, "m2_2p7b": 400, "m2_2p7b_16": 400, "hyb8b": 200,
+            "serve64": 30, "wide256": 30, "wide256_chain": 20}.get(name, 50)
+
+
+# ----------------------------------------------------------------------------- accounting
+
+
+def algorithmic_bytes(w):
+    """Bytes of one fused scan + commit launch (one layer): every tensor moved once."""
+    b, T, H, P, N, G = w.batch, w.n_nodes, w.nheads, w.headdim, w.dstate, w.ngroups
+    e = 2 if w.dtype == "bf16" else 4
+    state = b * H * P * N * 4
+    xy = b * T * H * P * e
+    return {
+        "h0": state, "h_new": state, "x": xy, "y": xy, "dt": b * T * H * e,
+        "B": b * T * G * N * e, "C": b * T * G * N * e, "A": H * 4, "D": H * 4,
+        "parent": b * T * 4, "path": b * w.maxlen * 4 + b * 4,
+    }
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(kernel_name):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu summary,
+    if that summary was taken on the current kernel source; else None."""
+    import hashlib
+    summ = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(summ):
+        return None
+    want = None
+    for line in open(summ):
+        if line.startswith("traffic:"):
+            kv = dict(t.split("=", 1) for t in line[len("traffic:"):].split())
+            want = kv
+    if not want or want.get("kernel") != kernel_name:
+        return None
+    src = os.path.join(ROOT, "hybrid_packed_tree_b200", "csrc", want.get("file", ""))
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if sha != want.get("sha"):
+        return None
+    return float(want["bytes_per_launch"])
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.strip().split(",") for r in self.file.read().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for nm, v in zip(names, r[5:9]):
+                    if "Active" in v and "Not" not in v:
+                        reasons.add(nm)
+            except Exception:
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+
+def dev_tensor(torch, a, io, device):
+    if io == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_packed_tree_b200 import stree
+    from hybrid_packed_tree_b200 import workloads as wl
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    w = wl.make_workload(args.config)
+    K = args.steps or default_steps(args.config)
+    Wm = max(3, args.warmup)
+    nl = w.nlayers
+    io = w.dtype
+
+    per_launch = algorithmic_bytes(w)
+    launch_bytes = sum(per_launch.values())
+    step_bytes = launch_bytes * nl
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nsets = max(1, -(-3 * l2 // step_bytes))          # rotated copies: > 3x L2 per cycle
+
+    # Device buffers: nsets copies of every layer's inputs and outputs.
+    sets = []
+    for s in range(nsets):
+        layers = []
+        for li in range(nl):
+            L = w.layers[li]
+            d = {k: dev_tensor(torch, getattr(L, k), io, device) for k in ("x", "dt", "B", "C")}
+            d.update({k: dev_tensor(torch, getattr(L, k), "f32", device) for k in ("A", "D", "h0")})
+            d["y"] = torch.empty_like(d["x"])
+            d["h_new"] = torch.empty_like(d["h0"])
+            layers.append(d)
+        tree = {"parent": torch.from_numpy(w.parent).to(device), "path": torch.from_numpy(w.path).to(device),
+                "path_len": torch.from_numpy(w.path_len).to(device)}
+        sets.append((layers, tree))
+
+    ctx = stree.stree_ctx_create()
+    stree.stree_ctx_set_kernel(ctx, args.kernel)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i, ev=None):
+        layers, tree = sets[i % nsets]
+        stree.stree_build_tree(ctx, tree["parent"], stream=stream)
+        for li, d in enumerate(layers):
+            if ev is not None:
+                ev[li][0].record(stream)
+            stree.stree_tree_scan_commit(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], None,
+                                         tree["path"], tree["path_len"], d["y"], d["h_new"], stream=stream)
+            if ev is not None:
+                ev[li][1].record(stream)
+
+    for i in range(Wm):
+        step(i)
+    stree.stree_sync_check(ctx, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # Timed region 1: the step time (value).
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(device)
+    n0 = stree.stree_ctx_launch_count(ctx)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    launches = stree.stree_ctx_launch_count(ctx) - n0
+    ms = t0.elapsed_time(t1)
+
+    # Timed region 2: the same steps with events around every fused launch
+    # (the dominant kernel's average launch duration for the roofline).
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nl)]
+           for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(device)
+    for i in range(K):
+        step(i, evs[i])
+    torch.cuda.synchronize(device)
+    barrier()
+    clk = clocks.stop()
+    kern_ms = [e[0].elapsed_time(e[1]) for per in evs for e in per]
+    st, info = stree.stree_sync_check(ctx, stream, raise_on_error=False)
+    if st != 0:
+        raise RuntimeError(f"device error during the benchmark: {info}")
+
+    if world > 1:
+        t = torch.tensor([ms, statistics.mean(kern_ms)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, kmean = float(t[0]), float(t[1])
+    else:
+        kmean = statistics.mean(kern_ms)
+
+    nodes_step = w.batch * w.n_nodes * nl
+    value = world * nodes_step * K / (ms / 1e3)
+    hbm_gbs, peak_kind = peaks()
+    achieved = launch_bytes / (kmean / 1e3) / 1e9
+    kernel_name = "scan_tc_kernel" if args.kernel != "simt" else "scan_simt_kernel"
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if io == "bf16" else "f32", "data": "synthetic (seeded; shapes and distributions of the workload)",
+        "config": {
+            "workload": args.config, "batch": w.batch, "layers": nl, "n_nodes": w.n_nodes, "nheads": w.nheads,
+            "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "io_dtype": io, "state_dtype": "f32",
+            "kernel": args.kernel, "parallelism": f"replicas x{world}",
+            "l2": f"rotates {nsets} buffer copies ({nsets * step_bytes / 2**20:.0f} MiB > 3x L2)"
+                  if nsets > 1 else "step bytes exceed L2 (no reuse between steps)",
+        },
+        "hbm": {"step_bytes": step_bytes, "gbs_step": step_bytes * K / (ms / 1e3) / 1e9},
+        "sequences_per_s": world * w.batch * K / (ms / 1e3),
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+            "frac": achieved / hbm_gbs, "traffic": profile_traffic(kernel_name),
+            "peak_source": f"{peak_kind} hbm_gbs", "kernel": kernel_name,
+            "bytes_per_launch": launch_bytes, "kernel_ms_mean": kmean,
+            "kernel_ms_median": statistics.median(kern_ms),
+        },
+        "clocks": clk,
+        "gpu_launches": int(launches),
+    }
+
+    if not args.no_e2e:
+        out["e2e"] = e2e(torch, stree, w, ctx, device, stream, args, world)
+    stree.stree_ctx_destroy(ctx)
+    return out
+
+
+def e2e(torch, stree, w, ctx, device, stream, args, world):
+    """Same metric through the public API with pinned host buffers: H2D of every
+    input of the step, the calls, D2H of y and h_new, all inside the timed region."""
+    import torch.distributed as dist
+    io = w.dtype
+    host_layers = []
+    for L in w.layers:
+        hl = {}
+        for k in ("x", "dt", "B", "C", "A", "D", "h0"):
+            t = dev_tensor(torch, getattr(L, k), io if k in ("x", "dt", "B", "C") else "f32", "cpu")
+            hl[k] = t.pin_memory()
+        hl["y"] = torch.empty_like(hl["x"]).pin_memory()
+        hl["h_new"] = torch.empty_like(hl["h0"]).pin_memory()
+        host_layers.append(hl)
+    htree = {k: torch.from_numpy(getattr(w, k)).pin_memory() for k in ("parent", "path", "path_len")}
+    dl = [{k: torch.empty_like(v, device=device) for k, v in hl.items()} for hl in host_layers]
+    dtree = {k: torch.empty_like(v, device=device) for k, v in htree.items()}
+    h2d = sum(v.numel() * v.element_size() for hl in host_layers for k, v in hl.items() if k not in ("y", "h_new"))
+    h2d += sum(v.numel() * v.element_size() for v in htree.values())
+    d2h = sum(hl[k].numel() * hl[k].element_size() for hl in host_layers for k in ("y", "h_new"))
+
+    def step():
+        for k in dtree:
+            dtree[k].copy_(htree[k], non_blocking=True)
+        stree.stree_build_tree(ctx, dtree["parent"], stream=stream)
+        for hl, d in zip(host_layers, dl):
+            for k in ("x", "dt", "B", "C", "A", "D", "h0"):
+                d[k].copy_(hl[k], non_blocking=True)
+            stree.stree_tree_scan_commit(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], None,
+                                         dtree["path"], dtree["path_len"], d["y"], d["h_new"], stream=stream)
+            hl["y"].copy_(d["y"], non_blocking=True)
+            hl["h_new"].copy_(d["h_new"], non_blocking=True)
+
+    K = max(3, min(args.steps or default_steps(args.config), 50 if w.nlayers * w.batch < 64 else 5))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    nodes = w.batch * w.n_nodes * w.nlayers
+    return {"value": world * nodes * K / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": K}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+
+def oracle_sample(name):
+    """A bounded sample of the workload for the CPU oracle: its first layer and at
+    most 8 sequences.  Returns (workload, description)."""
+    from hybrid_packed_tree_b200 import workloads as wl
+    b0 = wl.SPECS[name][1]
+    nb = min(b0, 8 if name not in ("wide256", "wide256_chain") else 2)
+    w = wl.make_workload(name, batch=nb, layers=1)
+    return w, f"layer 0 of {name}, {nb} of {b0} sequence(s), full heads and tree; scan + commit"
+
+
+def oracle_step(w, nthreads):
+    from oracle import oracle_commit, oracle_tree_scan
+    f = w.f64(0)
+    oracle_tree_scan(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["h0"], w.parent, nthreads=nthreads)
+    oracle_commit(f["x"], f["dt"], f["A"], f["B"], f["h0"], w.parent, w.path, w.path_len, nthreads=nthreads)
+
+
+def cpu_baseline(name, seconds):
+    from oracle.walk import default_threads
+    w, desc = oracle_sample(name)
+    cores = default_threads()
+    oracle_step(w, cores)                      # compile + warm
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(w, cores)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    nodes = w.batch * w.n_nodes * n
+    return {"value": nodes / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{desc}; {n} repetitions in {el:.1f} s on {cores} threads (fp64 root-path walk)"}
+
+
+def run_reference(args):
+    from oracle.walk import default_threads
+    w, desc = oracle_sample(args.config)
+    cores = default_threads()
+    K = args.steps or 3
+    Wm = max(3, args.warmup)
+    # Each step is one oracle pass over the bounded sample.
+    for _ in range(min(Wm, 3)):
+        oracle_step(w, cores)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        oracle_step(w, cores)
+    el = time.perf_counter() - t0
+    value = w.batch * w.n_nodes * K / el
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": K,
+        "warmup": Wm, "ms_per_step": el * 1e3 / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": args.config, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,67 @@
+"""Build ``libstree.so`` (the C ABI of include/stree.h) in-tree with nvcc for sm_100a.
+
+    python -m hybrid_packed_tree_b200.build [--force] [--debug]
+
+The library is written next to this file so that it travels with the source
+tree; nothing is installed into site-packages.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libstree.so")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def sources() -> list:
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
+def _deps() -> list:
+    return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+
+
+def is_stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    return any(os.path.getmtime(p) > t for p in _deps())
+
+
+def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
+    """Compile every .cu under csrc/ into libstree.so; returns its path."""
+    if not force and not debug and not is_stale():
+        return LIB
+    nvcc = os.environ.get("NVCC", "nvcc")
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc, *ARCH, "-lineinfo", "-O3", "-std=c++17",
+           "-cudart", "static", "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-o", tmp, *sources()]
+    if debug:
+        cmd.insert(1, "-DSTREE_DEBUG")
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--debug", action="store_true")
+    ap.add_argument("--verbose", action="store_true", help="pass -Xptxas=-v (registers, spills)")
+    args = ap.parse_args(argv)
+    print(build(force=args.force, debug=args.debug, verbose=args.verbose))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

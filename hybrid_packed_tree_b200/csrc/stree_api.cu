@@ -1,0 +1,317 @@
+// stree_api.cu -- the C ABI of include/stree.h: argument checks, the context's
+// workspace and the dispatch to the kernels.  No call here synchronises the
+// device except stree_sync_check and stree_ctx_destroy.
+#include <new>
+#include <string.h>
+
+#include "stree_internal.cuh"
+
+using namespace stree;
+
+struct stree_ctx {
+    int device = -1;
+    stree_kernel kernel = STREE_KERNEL_AUTO;
+    // tree workspace
+    uint32_t *anc = nullptr;
+    int32_t *depth = nullptr, *ok = nullptr;
+    size_t cap_anc = 0, cap_nodes = 0, cap_batch = 0;
+    int tree_T = 0, tree_batch = -1;
+    // C.B pair scratch
+    float *cb = nullptr;
+    size_t cap_cb = 0;
+    // error word {status, sequence, position, detail}
+    int32_t *err = nullptr;
+    // inputs recorded by the last scan, for stree_commit
+    bool has_scan = false;
+    ScanArgs last{};
+    int64_t launches = 0;
+};
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+stree_status cuda_status(cudaError_t e) { return e == cudaSuccess ? STREE_OK : STREE_ERR_CUDA; }
+
+template <typename T>
+stree_status ensure(T **buf, size_t *cap, size_t need)
+{
+    if (need <= *cap) return STREE_OK;
+    if (*buf) cudaFree(*buf);
+    *buf = nullptr;
+    *cap = 0;
+    if (cudaMalloc(reinterpret_cast<void **>(buf), need * sizeof(T)) != cudaSuccess) {
+        *buf = nullptr;
+        return STREE_ERR_CUDA;
+    }
+    *cap = need;
+    return STREE_OK;
+}
+
+TreeView tree_view(const stree_ctx *c)
+{
+    TreeView tv;
+    tv.anc = c->anc;
+    tv.depth = c->depth;
+    tv.ok = c->ok;
+    tv.T = c->tree_T;
+    tv.W = (c->tree_T + 31) / 32;
+    tv.batch = c->tree_batch;
+    return tv;
+}
+
+stree_status build_into_ctx(stree_ctx *c, const int32_t *parent, int T, int batch, cudaStream_t s)
+{
+    if (!parent) return STREE_ERR_INVALID_ARG;
+    if (T < 1 || T > kMaxNodes || batch < 0) return STREE_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(parent) & 3u) != 0) return STREE_ERR_MISALIGNED;
+    size_t W = (T + 31) / 32;
+    size_t nb = batch > 0 ? (size_t)batch : 1;
+    stree_status st;
+    if ((st = ensure(&c->anc, &c->cap_anc, nb * T * W)) != STREE_OK) return st;
+    if ((st = ensure(&c->depth, &c->cap_nodes, nb * T)) != STREE_OK) return st;
+    if ((st = ensure(&c->ok, &c->cap_batch, nb)) != STREE_OK) return st;
+    c->tree_T = T;
+    c->tree_batch = batch;
+    if (batch > 0) ++c->launches;
+    return cuda_status(launch_build_tree(parent, T, batch, c->anc, c->depth, c->ok, c->err, s));
+}
+
+stree_status check_scan_args(const ScanArgs &a)
+{
+    if (!a.x || !a.dt || !a.A || !a.B || !a.C || !a.D || !a.h0 || !a.y) return STREE_ERR_INVALID_ARG;
+    if (a.batch < 0 || a.T < 1 || a.H < 1 || a.G < 1 || a.P < 1 || a.N < 1) return STREE_ERR_UNSUPPORTED;
+    if (a.T > kMaxNodes || a.P > kMaxDim || a.N > kMaxDim) return STREE_ERR_UNSUPPORTED;
+    if (a.P % 8 != 0 || a.N % 8 != 0 || a.H % a.G != 0) return STREE_ERR_UNSUPPORTED;
+    if (a.H > 65535) return STREE_ERR_UNSUPPORTED;
+    if (a.dtype != STREE_F32 && a.dtype != STREE_BF16) return STREE_ERR_UNSUPPORTED;
+    const void *ptrs[] = {a.x, a.dt, a.A, a.B, a.C, a.D, a.h0, a.y};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return STREE_ERR_MISALIGNED;
+    return STREE_OK;
+}
+
+stree_status check_commit_args(const int32_t *path, const int32_t *path_len, int maxlen, const float *h_new)
+{
+    if (!path || !path_len || !h_new) return STREE_ERR_INVALID_ARG;
+    if (maxlen < 1) return STREE_ERR_INVALID_ARG;
+    if (!aligned16(h_new)) return STREE_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(path) & 3u) || (reinterpret_cast<uintptr_t>(path_len) & 3u))
+        return STREE_ERR_MISALIGNED;
+    return STREE_OK;
+}
+
+// Runs the scan (and the commit, when a.path is set) for a tree already in the ctx.
+stree_status run_scan(stree_ctx *c, ScanArgs &a, cudaStream_t s)
+{
+    if (c->tree_batch != a.batch || c->tree_T != a.T) return STREE_ERR_NO_TREE;
+    a.tree = tree_view(c);
+    a.err = c->err;
+    if (a.batch == 0) return STREE_OK;
+    bool use_tc = false;
+    if (c->kernel == STREE_KERNEL_TC) {
+        if (!tc_supported(a)) return STREE_ERR_UNSUPPORTED;
+        use_tc = true;
+    } else if (c->kernel == STREE_KERNEL_AUTO) {
+        use_tc = tc_supported(a);
+    }
+    if (use_tc) {
+        ++c->launches;
+        return cuda_status(launch_scan_tc(a, s));
+    }
+    stree_status st = ensure(&c->cb, &c->cap_cb, (size_t)a.batch * a.G * a.T * a.T);
+    if (st != STREE_OK) return st;
+    a.cb = c->cb;
+    if (a.y) {
+        ++c->launches;
+        if ((st = cuda_status(launch_cb_pairs(a, s))) != STREE_OK) return st;
+    }
+    ++c->launches;
+    return cuda_status(launch_scan_simt(a, s));
+}
+
+ScanArgs make_args(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                   const float *D, const float *h0, int T, int batch, int H, int P, int N, int G,
+                   stree_dtype dtype, void *y)
+{
+    ScanArgs a{};
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.h0 = h0;
+    a.T = T; a.batch = batch; a.H = H; a.P = P; a.N = N; a.G = G;
+    a.dtype = dtype;
+    a.y = y;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+stree_status stree_ctx_create(stree_ctx **out)
+{
+    if (!out) return STREE_ERR_INVALID_ARG;
+    *out = nullptr;
+    stree_ctx *c = new (std::nothrow) stree_ctx();
+    if (!c) return STREE_ERR_CUDA;
+    if (cudaGetDevice(&c->device) != cudaSuccess ||
+        cudaMalloc(reinterpret_cast<void **>(&c->err), 4 * sizeof(int32_t)) != cudaSuccess ||
+        cudaMemset(c->err, 0, 4 * sizeof(int32_t)) != cudaSuccess) {
+        if (c->err) cudaFree(c->err);
+        delete c;
+        return STREE_ERR_CUDA;
+    }
+    *out = c;
+    return STREE_OK;
+}
+
+stree_status stree_ctx_destroy(stree_ctx *c)
+{
+    if (!c) return STREE_OK;
+    cudaDeviceSynchronize();
+    cudaFree(c->anc);
+    cudaFree(c->depth);
+    cudaFree(c->ok);
+    cudaFree(c->cb);
+    cudaFree(c->err);
+    delete c;
+    return STREE_OK;
+}
+
+stree_status stree_ctx_set_kernel(stree_ctx *c, stree_kernel k)
+{
+    if (!c) return STREE_ERR_INVALID_ARG;
+    if (k != STREE_KERNEL_AUTO && k != STREE_KERNEL_SIMT && k != STREE_KERNEL_TC) return STREE_ERR_INVALID_ARG;
+    c->kernel = k;
+    return STREE_OK;
+}
+
+stree_status stree_ctx_launch_count(stree_ctx *c, int64_t *count)
+{
+    if (!c || !count) return STREE_ERR_INVALID_ARG;
+    *count = c->launches;
+    return STREE_OK;
+}
+
+stree_status stree_build_tree(stree_ctx *c, const int32_t *parent, int n_nodes, int batch,
+                              uint32_t *anc_out, int32_t *depth_out, void *stream)
+{
+    if (!c) return STREE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    stree_status st = build_into_ctx(c, parent, n_nodes, batch, s);
+    if (st != STREE_OK) return st;
+    size_t W = (n_nodes + 31) / 32;
+    if (anc_out && batch > 0)
+        if (cudaMemcpyAsync(anc_out, c->anc, (size_t)batch * n_nodes * W * sizeof(uint32_t),
+                            cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return STREE_ERR_CUDA;
+    if (depth_out && batch > 0)
+        if (cudaMemcpyAsync(depth_out, c->depth, (size_t)batch * n_nodes * sizeof(int32_t),
+                            cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return STREE_ERR_CUDA;
+    return STREE_OK;
+}
+
+stree_status stree_tree_scan(stree_ctx *c, const void *x, const void *dt, const float *A,
+                             const void *B, const void *C, const float *D, const float *h0,
+                             const int32_t *parent, int n_nodes, int batch, int nheads,
+                             int headdim, int dstate, int ngroups, stree_dtype dtype,
+                             void *y, void *stream)
+{
+    if (!c) return STREE_ERR_INVALID_ARG;
+    ScanArgs a = make_args(x, dt, A, B, C, D, h0, n_nodes, batch, nheads, headdim, dstate, ngroups, dtype, y);
+    stree_status st = check_scan_args(a);
+    if (st != STREE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (parent && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
+    if ((st = run_scan(c, a, s)) != STREE_OK) return st;
+    c->last = a;
+    c->has_scan = true;
+    return STREE_OK;
+}
+
+stree_status stree_commit(stree_ctx *c, const int32_t *path, const int32_t *path_len, int maxlen,
+                          float *h_new, void *stream)
+{
+    if (!c) return STREE_ERR_INVALID_ARG;
+    stree_status st = check_commit_args(path, path_len, maxlen, h_new);
+    if (st != STREE_OK) return st;
+    if (!c->has_scan) return STREE_ERR_NO_TREE;
+    ScanArgs a = c->last;
+    a.y = nullptr;
+    a.path = path;
+    a.path_len = path_len;
+    a.maxlen = maxlen;
+    a.h_new = h_new;
+    if (c->tree_batch != a.batch || c->tree_T != a.T) return STREE_ERR_NO_TREE;
+    a.tree = tree_view(c);
+    a.err = c->err;
+    if (a.batch == 0) return STREE_OK;
+    ++c->launches;
+    return cuda_status(launch_scan_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
+stree_status stree_tree_scan_commit(stree_ctx *c, const void *x, const void *dt, const float *A,
+                                    const void *B, const void *C, const float *D, const float *h0,
+                                    const int32_t *parent, int n_nodes, int batch, int nheads,
+                                    int headdim, int dstate, int ngroups, stree_dtype dtype,
+                                    const int32_t *path, const int32_t *path_len, int maxlen,
+                                    void *y, float *h_new, void *stream)
+{
+    if (!c) return STREE_ERR_INVALID_ARG;
+    ScanArgs a = make_args(x, dt, A, B, C, D, h0, n_nodes, batch, nheads, headdim, dstate, ngroups, dtype, y);
+    stree_status st = check_scan_args(a);
+    if (st != STREE_OK) return st;
+    if ((st = check_commit_args(path, path_len, maxlen, h_new)) != STREE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (parent && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
+    ScanArgs rec = a;
+    a.path = path;
+    a.path_len = path_len;
+    a.maxlen = maxlen;
+    a.h_new = h_new;
+    if ((st = run_scan(c, a, s)) != STREE_OK) return st;
+    c->last = rec;
+    c->has_scan = true;
+    return STREE_OK;
+}
+
+stree_status stree_resolve_path(stree_ctx *c, const int32_t *path, const int32_t *path_len, int maxlen,
+                                int32_t *leaf_out, void *stream)
+{
+    if (!c || !path || !path_len || !leaf_out || maxlen < 1) return STREE_ERR_INVALID_ARG;
+    if (c->tree_batch < 0) return STREE_ERR_NO_TREE;
+    if (c->tree_batch > 0) ++c->launches;
+    return cuda_status(launch_resolve_path(tree_view(c), path, path_len, maxlen, leaf_out, c->err,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+stree_status stree_sync_check(stree_ctx *c, void *stream, int32_t *info)
+{
+    if (!c) return STREE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t h[4] = {0, 0, 0, 0};
+    if (cudaStreamSynchronize(s) != cudaSuccess) return STREE_ERR_CUDA;
+    if (cudaMemcpy(h, c->err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return STREE_ERR_CUDA;
+    if (cudaMemset(c->err, 0, sizeof(h)) != cudaSuccess) return STREE_ERR_CUDA;
+    if (info) memcpy(info, h, sizeof(h));
+    return static_cast<stree_status>(h[0]);
+}
+
+const char *stree_status_string(stree_status st)
+{
+    switch (st) {
+    case STREE_OK: return "ok";
+    case STREE_ERR_INVALID_ARG: return "invalid argument";
+    case STREE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case STREE_ERR_BAD_TREE: return "parent array is not a packed tree";
+    case STREE_ERR_BAD_PATH: return "accepted path is not a root->node chain of the tree";
+    case STREE_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case STREE_ERR_CUDA: return "CUDA runtime error";
+    case STREE_ERR_TIMEOUT: return "device wait timed out";
+    case STREE_ERR_NO_TREE: return "no tree or scan recorded for these sizes";
+    }
+    return "unknown status";
+}
+
+int stree_version(void) { return 100; }
+
+}  // extern "C"

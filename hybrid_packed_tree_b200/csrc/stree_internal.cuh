@@ -1,0 +1,74 @@
+// stree_internal.cuh -- types shared by the libstree translation units.
+//
+// Nothing here is part of the C ABI (include/stree.h is).  The context owns the
+// device workspace; kernels receive plain pointers through ScanArgs.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "stree.h"
+
+namespace stree {
+
+constexpr int kMaxNodes = 256;                 // n_nodes limit (mask words <= 8)
+constexpr int kMaxWords = kMaxNodes / 32;
+constexpr int kMaxDim = 256;                   // headdim / dstate limit
+
+// Device error word: {status, sequence, position, detail}.  The first error wins.
+__device__ __forceinline__ void latch_error(int32_t *err, int code, int b, int pos, int detail)
+{
+    if (atomicCAS(err, 0, code) == 0) {
+        err[1] = b;
+        err[2] = pos;
+        err[3] = detail;
+    }
+}
+
+struct TreeView {
+    const uint32_t *anc;     // [batch, T, W]
+    const int32_t *depth;    // [batch, T]
+    const int32_t *ok;       // [batch]
+    int T, W, batch;
+};
+
+struct ScanArgs {
+    const void *x, *dt, *B, *C;
+    const float *A, *D, *h0;
+    int T, batch, H, P, N, G;
+    stree_dtype dtype;
+    void *y;                           // NULL: no outputs y (commit only)
+    const int32_t *path, *path_len;    // NULL path: no commit
+    int maxlen;
+    float *h_new;
+    TreeView tree;
+    float *cb;                         // scratch [batch, G, T, T]: C_i . B_j on ancestor pairs
+    int32_t *err;
+};
+
+// Kernel launchers (each returns cudaSuccess or the launch error).
+cudaError_t launch_build_tree(const int32_t *parent, int T, int batch, uint32_t *anc, int32_t *depth,
+                              int32_t *ok, int32_t *err, cudaStream_t s);
+cudaError_t launch_resolve_path(const TreeView &tv, const int32_t *path, const int32_t *path_len,
+                                int maxlen, int32_t *leaf_out, int32_t *err, cudaStream_t s);
+cudaError_t launch_cb_pairs(const ScanArgs &a, cudaStream_t s);
+cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t s);
+
+// Tensor-core path: whether the shape is supported, and the launcher.
+bool tc_supported(const ScanArgs &a);
+cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
+
+__device__ __forceinline__ float load_as_float(const void *p, size_t i, stree_dtype dt)
+{
+    if (dt == STREE_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ void store_from_float(void *p, size_t i, float v, stree_dtype dt)
+{
+    if (dt == STREE_BF16) reinterpret_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+    else reinterpret_cast<float *>(p)[i] = v;
+}
+
+}  // namespace stree

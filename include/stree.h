@@ -1,0 +1,174 @@
+/*
+ * stree.h -- C ABI of libstree.so: the packed-tree selective-SSM scan on B200.
+ *
+ * The method ("STree: Speculative Tree Decoding for Hybrid State Space Models",
+ * scime.ai summary, sections "Problem" and "Approach"): a speculative draft tree
+ * is packed into one sequence with a tree mask; accumulating the diagonal log
+ * state transitions along each node's ancestors (A_tree = L . log A) gives the
+ * exact per-path SSM output of every node in one scan, and after acceptance the
+ * state of the accepted path is rebuilt from the stored inputs ("activation
+ * replay") instead of keeping per-node states.  The same replay-on-commit design
+ * appears in "Bole" (abstract: reconstruct only the selected state) and "TreeWY"
+ * (abstract: reconstruct only the accepted state on commit).
+ *
+ * Per sequence b, head h (group g = h / (H/G)) and node i with parent p(i):
+ *     s_i = exp(dt_i A_h) s_p(i) + dt_i x_i (outer) B_i,   s_p(root) = h0[b,h]
+ *     y_i = s_i C_i + D_h x_i
+ * computed in packed form as
+ *     L_i = A_h * sum_{j in anc(i)} dt_j                      (tree cumsum)
+ *     y_i = exp(L_i) (h0 C_i) + sum_{j in anc(i)} exp(L_i - L_j) (C_i . B_j) dt_j x_j + D_h x_i
+ * and the commit of an accepted root->leaf path as
+ *     h_new = exp(L_leaf) h0 + sum_{j on path} exp(L_leaf - L_j) dt_j x_j (outer) B_j.
+ * anc(i) is the ancestor-or-self set of i.  dt is taken as given (already passed
+ * through softplus); there is no dt bias, gating or normalisation in this op.
+ *
+ * Layouts (contiguous, row-major, device memory unless stated):
+ *   x     [batch, n_nodes, nheads, headdim]   dtype (fp32 or bf16)
+ *   dt    [batch, n_nodes, nheads]            dtype
+ *   A, D  [nheads]                            fp32
+ *   B, C  [batch, n_nodes, ngroups, dstate]   dtype
+ *   h0    [batch, nheads, headdim, dstate]    fp32 (the cached state)
+ *   y     [batch, n_nodes, nheads, headdim]   dtype
+ *   h_new [batch, nheads, headdim, dstate]    fp32
+ *   parent [batch, n_nodes] int32: parent[b,0] = -1 and 0 <= parent[b,i] < i
+ *          for i > 0 (the tree is packed in a topological order, root first).
+ *   accepted_path [batch, maxlen] int32, path_len [batch] int32: path[b,0] = 0
+ *          and parent[path[b,k]] = path[b,k-1]; entries past path_len ignored;
+ *          path_len = 0 keeps the cached state (h_new = h0).
+ *   anc   [batch, n_nodes, ceil(n_nodes/32)] uint32: bit j of word j/32 set iff
+ *          j is i or an ancestor of i.  depth [batch, n_nodes] int32 (root 0).
+ *
+ * Supported shapes: 1 <= n_nodes <= 256, batch >= 0, headdim and dstate multiples
+ * of 8 in [8, 256], nheads a multiple of ngroups.  Pointers to tensors must be
+ * 16-byte aligned.  batch = 0 is a no-op that returns STREE_OK.
+ *
+ * Ownership and threading: the caller owns every tensor.  A context (stree_ctx)
+ * owns the library's device workspace (tree masks, depths, per-sequence flags,
+ * the error word, a C.B scratch for the tree term).  Workspace is allocated by
+ * cudaMalloc the first time a call needs more than the context holds; later
+ * calls with the same or smaller sizes never allocate, so warm a context up
+ * before capturing its calls in a CUDA graph.  A context is not thread-safe;
+ * use one per stream.  All calls are asynchronous on `stream` (a cudaStream_t;
+ * NULL is the legacy default stream) except stree_sync_check and
+ * stree_ctx_destroy.
+ *
+ * Errors: every call returns a status and never aborts.  Argument and shape
+ * checks happen on the host before anything is launched.  Tree and path validity
+ * are checked on the device: a bad sequence is skipped (its outputs are left
+ * untouched) and the first such error is latched in the context's error word,
+ * which stree_sync_check reads and clears.
+ */
+#ifndef STREE_H
+#define STREE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    STREE_OK = 0,
+    STREE_ERR_INVALID_ARG = 1,  /* null pointer, negative size, aliasing not allowed */
+    STREE_ERR_UNSUPPORTED = 2,  /* shape or dtype outside the supported set */
+    STREE_ERR_BAD_TREE = 3,     /* device-detected: parent array is not a packed tree */
+    STREE_ERR_BAD_PATH = 4,     /* device-detected: accepted path is not a root->node chain */
+    STREE_ERR_MISALIGNED = 5,   /* a tensor pointer is not 16-byte aligned */
+    STREE_ERR_CUDA = 6,         /* a CUDA runtime call failed (launch, allocation) */
+    STREE_ERR_TIMEOUT = 7,      /* a bounded device wait gave up (reserved) */
+    STREE_ERR_NO_TREE = 8       /* scan with parent = NULL before any tree was built, or
+                                   commit before any scan, or a size mismatch with them */
+} stree_status;
+
+typedef enum { STREE_F32 = 0, STREE_BF16 = 1 } stree_dtype;
+
+/* Which scan kernel a context uses (stree_ctx_set_kernel). */
+typedef enum {
+    STREE_KERNEL_AUTO = 0,      /* tensor-core kernel where supported, else SIMT */
+    STREE_KERNEL_SIMT = 1,      /* CUDA-core fp32 kernel, every supported shape */
+    STREE_KERNEL_TC = 2         /* tcgen05 kernel; STREE_ERR_UNSUPPORTED if the shape is not */
+} stree_kernel;
+
+typedef struct stree_ctx stree_ctx;
+
+/* Create / destroy a context.  destroy synchronises the device and frees the
+ * workspace; it accepts NULL. */
+stree_status stree_ctx_create(stree_ctx **out);
+stree_status stree_ctx_destroy(stree_ctx *ctx);
+
+/* Select the scan kernel for later scan calls on this context (default AUTO). */
+stree_status stree_ctx_set_kernel(stree_ctx *ctx, stree_kernel kernel);
+
+/* Number of CUDA kernels this context has launched so far (host counter). */
+stree_status stree_ctx_launch_count(stree_ctx *ctx, int64_t *count);
+
+/*
+ * Tree builder ("tree mask" of the packed sequence, STree summary "Approach"):
+ * validates parent[] and builds the ancestor-or-self bitmask and depth of every
+ * node into the context.  anc_out / depth_out, when not NULL, receive copies
+ * (device buffers of the layouts above).  An invalid tree latches
+ * STREE_ERR_BAD_TREE and marks the sequence so that scans skip it.
+ */
+stree_status stree_build_tree(stree_ctx *ctx, const int32_t *parent, int n_nodes, int batch,
+                              uint32_t *anc_out, int32_t *depth_out, void *stream);
+
+/*
+ * Packed tree scan: y for every node of every sequence and head.  When parent is
+ * not NULL the tree is (re)built first (as stree_build_tree); when it is NULL
+ * the context's current tree is used and n_nodes / batch must match it.  The
+ * input pointers are recorded for a later stree_commit (activation replay), so
+ * x, dt, A, B and h0 must stay alive and unchanged until that commit.
+ */
+stree_status stree_tree_scan(stree_ctx *ctx, const void *x, const void *dt, const float *A,
+                             const void *B, const void *C, const float *D, const float *h0,
+                             const int32_t *parent, int n_nodes, int batch, int nheads,
+                             int headdim, int dstate, int ngroups, stree_dtype dtype,
+                             void *y, void *stream);
+
+/*
+ * Commit by activation replay (STree summary, "Approach"): h_new for the
+ * accepted path of every sequence, from the inputs recorded by the last
+ * stree_tree_scan on this context.  h_new may alias the recorded h0 (in-place
+ * commit); no other aliasing is allowed.  An invalid path latches
+ * STREE_ERR_BAD_PATH and leaves that sequence's h_new untouched.
+ */
+stree_status stree_commit(stree_ctx *ctx, const int32_t *accepted_path, const int32_t *path_len,
+                          int maxlen, float *h_new, void *stream);
+
+/*
+ * Fused scan + commit: y and h_new in one pass that reads h0 once.  Arguments as
+ * for stree_tree_scan followed by those of stree_commit.  h_new may alias h0.
+ */
+stree_status stree_tree_scan_commit(stree_ctx *ctx, const void *x, const void *dt, const float *A,
+                                    const void *B, const void *C, const float *D, const float *h0,
+                                    const int32_t *parent, int n_nodes, int batch, int nheads,
+                                    int headdim, int dstate, int ngroups, stree_dtype dtype,
+                                    const int32_t *accepted_path, const int32_t *path_len,
+                                    int maxlen, void *y, float *h_new, void *stream);
+
+/*
+ * Resolve accepted paths against the context's current tree: leaf_out[b] (device
+ * int32 [batch]) receives the last node of a valid path, -1 for an empty path and
+ * -2 for an invalid one (which also latches STREE_ERR_BAD_PATH).
+ */
+stree_status stree_resolve_path(stree_ctx *ctx, const int32_t *accepted_path, const int32_t *path_len,
+                                int maxlen, int32_t *leaf_out, void *stream);
+
+/*
+ * Synchronise `stream`, read and clear the context's device error word.  Returns
+ * the latched status (STREE_OK when none).  info, when not NULL, receives four
+ * host int32: status, sequence index, node or path position, detail.
+ */
+stree_status stree_sync_check(stree_ctx *ctx, void *stream, int32_t *info);
+
+/* Static text for a status code. */
+const char *stree_status_string(stree_status status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int stree_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STREE_H */
