@@ -62,8 +62,8 @@ TreeView tree_view(const stree_ctx *c)
 
 stree_status build_into_ctx(stree_ctx *c, const int32_t *parent, int T, int batch, cudaStream_t s)
 {
-    if (!parent) return STREE_ERR_INVALID_ARG;
     if (T < 1 || T > kMaxNodes || batch < 0) return STREE_ERR_UNSUPPORTED;
+    if (!parent && batch > 0) return STREE_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(parent) & 3u) != 0) return STREE_ERR_MISALIGNED;
     size_t W = (T + 31) / 32;
     size_t nb = batch > 0 ? (size_t)batch : 1;
@@ -79,8 +79,9 @@ stree_status build_into_ctx(stree_ctx *c, const int32_t *parent, int T, int batc
 
 stree_status check_scan_args(const ScanArgs &a)
 {
-    if (!a.x || !a.dt || !a.A || !a.B || !a.C || !a.D || !a.h0 || !a.y) return STREE_ERR_INVALID_ARG;
     if (a.batch < 0 || a.T < 1 || a.H < 1 || a.G < 1 || a.P < 1 || a.N < 1) return STREE_ERR_UNSUPPORTED;
+    if (a.batch == 0) return STREE_OK;             // no-op: empty tensors may have NULL data
+    if (!a.x || !a.dt || !a.A || !a.B || !a.C || !a.D || !a.h0 || !a.y) return STREE_ERR_INVALID_ARG;
     if (a.T > kMaxNodes || a.P > kMaxDim || a.N > kMaxDim) return STREE_ERR_UNSUPPORTED;
     if (a.P % 8 != 0 || a.N % 8 != 0 || a.H % a.G != 0) return STREE_ERR_UNSUPPORTED;
     if (a.H > 65535) return STREE_ERR_UNSUPPORTED;
@@ -91,8 +92,10 @@ stree_status check_scan_args(const ScanArgs &a)
     return STREE_OK;
 }
 
-stree_status check_commit_args(const int32_t *path, const int32_t *path_len, int maxlen, const float *h_new)
+stree_status check_commit_args(const int32_t *path, const int32_t *path_len, int maxlen, const float *h_new,
+                               int batch)
 {
+    if (batch == 0) return maxlen >= 0 ? STREE_OK : STREE_ERR_INVALID_ARG;
     if (!path || !path_len || !h_new) return STREE_ERR_INVALID_ARG;
     if (maxlen < 1) return STREE_ERR_INVALID_ARG;
     if (!aligned16(h_new)) return STREE_ERR_MISALIGNED;
@@ -115,10 +118,6 @@ stree_status run_scan(stree_ctx *c, ScanArgs &a, cudaStream_t s)
     } else if (c->kernel == STREE_KERNEL_AUTO) {
         use_tc = tc_supported(a);
     }
-    if (use_tc) {
-        ++c->launches;
-        return cuda_status(launch_scan_tc(a, s));
-    }
     stree_status st = ensure(&c->cb, &c->cap_cb, (size_t)a.batch * a.G * a.T * a.T);
     if (st != STREE_OK) return st;
     a.cb = c->cb;
@@ -127,6 +126,7 @@ stree_status run_scan(stree_ctx *c, ScanArgs &a, cudaStream_t s)
         if ((st = cuda_status(launch_cb_pairs(a, s))) != STREE_OK) return st;
     }
     ++c->launches;
+    if (use_tc) return cuda_status(launch_scan_tc(a, s));
     return cuda_status(launch_scan_simt(a, s));
 }
 
@@ -221,7 +221,7 @@ stree_status stree_tree_scan(stree_ctx *c, const void *x, const void *dt, const 
     stree_status st = check_scan_args(a);
     if (st != STREE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (parent && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
+    if ((parent || batch == 0) && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
     if ((st = run_scan(c, a, s)) != STREE_OK) return st;
     c->last = a;
     c->has_scan = true;
@@ -232,9 +232,9 @@ stree_status stree_commit(stree_ctx *c, const int32_t *path, const int32_t *path
                           float *h_new, void *stream)
 {
     if (!c) return STREE_ERR_INVALID_ARG;
-    stree_status st = check_commit_args(path, path_len, maxlen, h_new);
-    if (st != STREE_OK) return st;
     if (!c->has_scan) return STREE_ERR_NO_TREE;
+    stree_status st = check_commit_args(path, path_len, maxlen, h_new, c->last.batch);
+    if (st != STREE_OK) return st;
     ScanArgs a = c->last;
     a.y = nullptr;
     a.path = path;
@@ -260,9 +260,9 @@ stree_status stree_tree_scan_commit(stree_ctx *c, const void *x, const void *dt,
     ScanArgs a = make_args(x, dt, A, B, C, D, h0, n_nodes, batch, nheads, headdim, dstate, ngroups, dtype, y);
     stree_status st = check_scan_args(a);
     if (st != STREE_OK) return st;
-    if ((st = check_commit_args(path, path_len, maxlen, h_new)) != STREE_OK) return st;
+    if ((st = check_commit_args(path, path_len, maxlen, h_new, batch)) != STREE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (parent && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
+    if ((parent || batch == 0) && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
     ScanArgs rec = a;
     a.path = path;
     a.path_len = path_len;

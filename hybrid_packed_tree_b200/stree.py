@@ -48,9 +48,9 @@ _lib.stree_ctx_destroy.argtypes = [_vp]
 _lib.stree_ctx_set_kernel.argtypes = [_vp, _i]
 _lib.stree_ctx_launch_count.argtypes = [_vp, ctypes.POINTER(ctypes.c_int64)]
 _lib.stree_build_tree.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp]
-_lib.stree_tree_scan.argtypes = [_vp] * 9 + [_i] * 7 + [_i, _vp, _vp]
+_lib.stree_tree_scan.argtypes = [_vp] * 9 + [_i] * 7 + [_vp, _vp]
 _lib.stree_commit.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
-_lib.stree_tree_scan_commit.argtypes = [_vp] * 9 + [_i] * 7 + [_i, _vp, _vp, _i, _vp, _vp, _vp]
+_lib.stree_tree_scan_commit.argtypes = [_vp] * 9 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp]
 _lib.stree_resolve_path.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
 _lib.stree_sync_check.argtypes = [_vp, _vp, _ip]
 _lib.stree_status_string.argtypes = [_i]

@@ -80,3 +80,27 @@ def test_library_does_not_load_the_oracle(lib_path):
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", text, re.M), f
                 assert "liboracle" not in text and "stree_oracle" not in text, f
+
+
+def _decl_arg_counts():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(stree_[a-z_]+)\s*\(([^;{]*?)\)\s*;", text):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_header(lib_path):
+    """Every binding prototype has the header's argument count, and a NULL context
+    is rejected on the host with STREE_ERR_INVALID_ARG (no device work)."""
+    from hybrid_packed_tree_b200 import stree
+    counts = _decl_arg_counts()
+    assert set(counts) == set(stree.EXPORTS)
+    for name, n in counts.items():
+        fn = getattr(stree._lib, name)
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+        if name.startswith("stree_") and fn.argtypes and name not in (
+                "stree_status_string", "stree_ctx_create", "stree_ctx_destroy"):
+            args = [0 if t is ctypes.c_int else None for t in fn.argtypes]
+            assert fn(*args) == 1, name
