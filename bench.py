@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample budget")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
+    ap.add_argument("--layers", type=int, default=None, help="override the workload's layer count (profiling)")
     return ap.parse_args()
 
 
@@ -175,7 +177,7 @@ def run_ours(args, rank, world, local_rank):
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    w = wl.make_workload(args.config)
+    w = wl.make_workload(args.config, batch=args.batch, layers=args.layers)
     K = args.steps or default_steps(args.config)
     Wm = max(3, args.warmup)
     nl = w.nlayers

@@ -33,27 +33,41 @@
 namespace stree {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kDstate = 128;               // dstate of the tensor-core path
 constexpr int kMaxTcNodes = 128;           // T_pad <= 128 (TMEM columns, smem)
+constexpr int kDtBox = 16;                 // heads per dt box (32 bytes of bf16)
+constexpr int kPathRows = 16;              // accepted-path rows of B staged in smem
 constexpr size_t kSmemLimit = 232448;      // 227 KB opt-in dynamic shared memory
 
-enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, kMiscWords = 8 };
+enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_WSUM = 8, kMiscWords = 16 };
 
 struct TcParams {
-    const __nv_bfloat16 *dt, *B, *C;
-    const float *A, *D;
-    const int32_t *path, *path_len;
-    const float *cb;
+    const __nv_bfloat16 *__restrict__ B;
+    const __nv_bfloat16 *__restrict__ C;
+    const float *__restrict__ A;
+    const float *__restrict__ D;
+    const int32_t *__restrict__ path;
+    const int32_t *__restrict__ path_len;
     TreeView tree;
     int32_t *err;
-    int T, T_pad, H, P, G, RB, tps, ntiles, maxlen, do_commit, hpt, pair_cap;
+    int T, T_pad, KA, H, P, G, RB, NB, tps, ntiles, maxlen, do_commit, hpt, pair_cap, dt_box;
     uint32_t tmem_cols;
-    uint32_t off_x, x_stage, off_c, off_anc, off_poff, off_dts, off_L, off_eL, off_w, off_alpha, off_pnode,
-        off_bar, off_misc, off_pcb, off_pj;
+    uint32_t off_x, x_dt, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_dts, off_L, off_eL,
+        off_w, off_alpha, off_pnode, off_bar, off_misc, off_pcb, off_pj;
 };
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+__device__ __forceinline__ void unpack4(uint2 raw, float &a, float &b, float &c, float &d)
+{
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
+    a = __low2float(lo);
+    b = __high2float(lo);
+    c = __low2float(hi);
+    d = __high2float(hi);
+}
 
 __device__ __forceinline__ int nth_set_bit(const uint32_t *row, int W, int n)
 {
@@ -65,20 +79,97 @@ __device__ __forceinline__ int nth_set_bit(const uint32_t *row, int W, int n)
     return -1;
 }
 
+// C_i . B_j: C from the staged fp32 MMA operand (swizzled), B_j from global memory.
+__device__ __forceinline__ float dot_cb(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i)
+{
+    float acc = 0.f;
+    const uint8_t *crow = cs + i * 128;
+    const uint2 *brow = reinterpret_cast<const uint2 *>(Bj);
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {
+        const float4 cv = *reinterpret_cast<const float4 *>(crow + (c >> 3) * T_pad * 128 + (((c & 7) ^ (i & 7)) << 4));
+        float b0, b1, b2, b3;
+        unpack4(__ldg(brow + c), b0, b1, b2, b3);
+        acc = fmaf(cv.x, b0, acc);
+        acc = fmaf(cv.y, b1, acc);
+        acc = fmaf(cv.z, b2, acc);
+        acc = fmaf(cv.w, b3, acc);
+    }
+    return acc;
+}
+
+// Byte offset of bf16 element (k row, m column) in an MN-major 128-byte swizzled
+// block stack: 64 columns per block, blocks `bstride` bytes apart.
+__device__ __forceinline__ uint32_t mn_off(int krow, int m, uint32_t bstride)
+{
+    return (uint32_t)(m >> 6) * bstride + (uint32_t)krow * 128u +
+           ((uint32_t)(((m & 63) >> 3) ^ (krow & 7)) << 4) + (uint32_t)(m & 7) * 2u;
+}
+
+// Byte offset of bf16 element (row, k) in a K-major 128-byte swizzled operand of
+// `rows` rows: 64 K-columns per atom, atoms rows*128 bytes apart.
+__device__ __forceinline__ uint32_t k_off(int row, int kcol, int rows)
+{
+    return (uint32_t)(kcol >> 6) * (uint32_t)rows * 128u + (uint32_t)row * 128u +
+           ((uint32_t)(((kcol & 63) >> 3) ^ (row & 7)) << 4) + (uint32_t)(kcol & 7) * 2u;
+}
+
+// Commit of one tile row segment: h_new = alpha h0 + sum_q coef_q B[pnode_q] (fp32).
+// The first kPathRows path rows of B come from shared memory, later ones from global.
+template <int CPT>
+__device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, uint32_t xbs, const __nv_bfloat16 *Bp,
+                                            const __nv_bfloat16 *Bseq, size_t brow_stride, const int16_t *pnode,
+                                            const float *wh, float al, int len, int RB, int row, int c_lo)
+{
+    float acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
+    for (int q = 0; q < len; ++q) {
+        const int j = pnode[q];
+        const float coef = wh[q] * bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + mn_off(j, row, xbs)));
+        const uint2 *src = q < kPathRows ? reinterpret_cast<const uint2 *>(Bp + q * kDstate + c_lo)
+                                         : reinterpret_cast<const uint2 *>(Bseq + (size_t)j * brow_stride + c_lo);
+#pragma unroll
+        for (int c = 0; c < CPT / 4; ++c) {
+            float b0, b1, b2, b3;
+            unpack4(src[c], b0, b1, b2, b3);
+            acc[4 * c + 0] = fmaf(coef, b0, acc[4 * c + 0]);
+            acc[4 * c + 1] = fmaf(coef, b1, acc[4 * c + 1]);
+            acc[4 * c + 2] = fmaf(coef, b2, acc[4 * c + 2]);
+            acc[4 * c + 3] = fmaf(coef, b3, acc[4 * c + 3]);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < CPT / 4; ++c) {
+        const int n = c_lo + 4 * c;
+        const int kb = n >> 5, ch = (n & 31) >> 2;
+        float4 *ptr = reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
+        float4 v = *ptr;
+        v.x = fmaf(al, v.x, acc[4 * c + 0]);
+        v.y = fmaf(al, v.y, acc[4 * c + 1]);
+        v.z = fmaf(al, v.z, acc[4 * c + 2]);
+        v.w = fmaf(al, v.w, acc[4 * c + 3]);
+        *ptr = v;
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant__ CUtensorMap tm_hn,
                const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
-               const TcParams p)
+               const __grid_constant__ CUtensorMap tm_dt, const TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int T = p.T, RB = p.RB, P = p.P, H = p.H, G = p.G, W = p.tree.W, HP = H * P;
+    const int T = p.T, T_pad = p.T_pad, RB = p.RB, P = p.P, H = p.H, G = p.G, W = p.tree.W, HP = H * P;
     const int hpg = H / G;
+    const uint32_t xbs = (uint32_t)T_pad * 128u;                      // x: bytes per 64-column block
 
-    uint8_t *h0s = smem;                                            // 2 x [4 atoms][RB rows][128 B]
-    uint8_t *xs = smem + p.off_x;                                   // 2 x [T][RB] bf16
-    uint8_t *cs = smem + p.off_c;                                   // [4 atoms][T_pad rows][128 B]
+    uint8_t *h0s = smem;                                              // 2 x [4 atoms][RB rows][128 B] fp32
+    uint8_t *xs = smem + p.off_x;                                     // 2 x {NB x [T_pad rows][128 B] x, dt}
+    uint8_t *cs = smem + p.off_c;                                     // [4 atoms][T_pad rows][128 B] fp32
+    uint8_t *mh = smem + p.off_mh;                                    // hpt x [KA atoms][T_pad rows][128 B] bf16
+    __nv_bfloat16 *Bp = reinterpret_cast<__nv_bfloat16 *>(smem + p.off_bp);  // [kPathRows][128]
     uint32_t *ancs = reinterpret_cast<uint32_t *>(smem + p.off_anc);  // [T][W]
     int32_t *poff = reinterpret_cast<int32_t *>(smem + p.off_poff);   // [T+1]
     float *dts = reinterpret_cast<float *>(smem + p.off_dts);         // [hpt][T]
@@ -95,12 +186,14 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     const uint32_t bar_full0 = ptx::smem_u32(&bars[0]);
     const uint32_t bar_mma = ptx::smem_u32(&bars[2]);
     const uint32_t h0_stage_bytes = (uint32_t)RB * 512u;
-    const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u;
-    const uint32_t idesc = ptx::idesc_tf32(128, p.T_pad);
+    const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u + (uint32_t)T * p.dt_box * 2u;
+    const uint32_t idesc_root = ptx::idesc_tf32(128, T_pad);
+    const uint32_t idesc_tree = ptx::idesc_bf16_amn(128, T_pad);
 
     if (tid == 0) {
         ptx::prefetch_tensormap(&tm_h0);
         ptx::prefetch_tensormap(&tm_x);
+        ptx::prefetch_tensormap(&tm_dt);
         ptx::prefetch_tensormap(&tm_hn);
         ptx::prefetch_tensormap(&tm_y);
         ptx::mbar_init(bar_full0, 1);
@@ -109,9 +202,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         ptx::fence_mbar_init();
         for (int k = 0; k < kMiscWords; ++k) misc[k] = 0;
     }
-    // Rows the MMA reads past an RB-row atom alias the next atom or the x
-    // region; give every byte a defined value once.
-    for (uint32_t o = tid * 16u; o < p.off_c; o += kThreads * 16u)
+    // Operand rows the MMAs read past the valid tile (rows >= RB, nodes >= T)
+    // must hold finite values: clear the staging regions once.
+    for (uint32_t o = tid * 16u; o < p.off_mh; o += kThreads * 16u)
         *reinterpret_cast<float4 *>(smem + o) = make_float4(0.f, 0.f, 0.f, 0.f);
     if (warp == 0) {
         ptx::tmem_alloc(ptx::smem_u32(&misc[M_TMEM]), p.tmem_cols);
@@ -132,12 +225,16 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     };
     auto issue_load = [&](int t, int stage) {
         const int b = t / p.tps, r0 = (t % p.tps) * RB;
+        const int hf8 = (r0 / P) & ~7;
         const uint32_t bar = bar_full0 + 8u * stage;
         ptx::mbar_expect_tx(bar, tx_bytes);
         const uint32_t dst = ptx::smem_u32(h0s + stage * h0_stage_bytes);
         for (int kb = 0; kb < 4; ++kb)
             ptx::tma_load_2d(dst + kb * RB * 128, &tm_h0, kb * 32, b * HP + r0, bar);
-        ptx::tma_load_2d(ptx::smem_u32(xs + stage * p.x_stage), &tm_x, r0, b * T, bar);
+        const uint32_t xdst = ptx::smem_u32(xs + stage * p.x_stage);
+        for (int nb = 0; nb < p.NB; ++nb)
+            ptx::tma_load_2d(xdst + nb * xbs, &tm_x, r0 + nb * 64, b * T, bar);
+        ptx::tma_load_2d(xdst + p.x_dt, &tm_dt, hf8, b * T, bar);
     };
 
     int t = next_valid(start);
@@ -152,12 +249,28 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         const int g = hfirst / hpg;
         const int key = b * G + g;
         const int stage = k & 1;
+        const __nv_bfloat16 *Bseq = p.B + ((size_t)b * T * G + g) * kDstate;   // row j at + j * G * 128
+        const size_t brow = (size_t)G * kDstate;
 
         // ---------------------------------------------------- per (sequence, group)
         if (key != cur_key) {
-            if (b != cur_b) {
+            const bool new_b = (b != cur_b);
+            for (int q = tid; q < T_pad * 32; q += kThreads) {
+                const int i = q >> 5, c = q & 31;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < T) {
+                    float c0, c1, c2, c3;
+                    unpack4(__ldg(reinterpret_cast<const uint2 *>(p.C + (((size_t)b * T + i) * G + g) * kDstate + c * 4)),
+                            c0, c1, c2, c3);
+                    v = make_float4(c0, c1, c2, c3);
+                }
+                const int kb = c >> 3, ch = c & 7;
+                *reinterpret_cast<float4 *>(cs + kb * T_pad * 128 + i * 128 + ((ch ^ (i & 7)) << 4)) = v;
+            }
+            if (new_b) {
                 for (int q = tid; q < T * W; q += kThreads) ancs[q] = __ldg(&p.tree.anc[(size_t)b * T * W + q]);
-                __syncthreads();
+                for (uint32_t o = tid * 16u; o < (uint32_t)p.hpt * p.mh_head; o += kThreads * 16u)
+                    *reinterpret_cast<float4 *>(mh + o) = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (tid == 0) {
                     int len = 0, state = 0;
                     if (p.do_commit) {
@@ -167,56 +280,68 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                             state = 0;
                             latch_error(p.err, STREE_ERR_BAD_PATH, b, -1, len);
                         } else if (len > 0) {
-                            const int32_t *pb = p.path + (size_t)b * p.maxlen;
-                            const int leaf = __ldg(&pb[len - 1]);
+                            const int leaf = __ldg(&p.path[(size_t)b * p.maxlen + len - 1]);
                             if (leaf < 0 || leaf >= T || __ldg(&p.tree.depth[(size_t)b * T + leaf]) != len - 1) {
                                 state = 0;
                                 latch_error(p.err, STREE_ERR_BAD_PATH, b, len - 1, leaf);
-                            } else {
-                                for (int q = 0; q < len; ++q) {
-                                    const int j = __ldg(&pb[q]);
-                                    const bool good = j >= 0 && j < T && ((ancs[leaf * W + (j >> 5)] >> (j & 31)) & 1u) &&
-                                                      __ldg(&p.tree.depth[(size_t)b * T + j]) == q;
-                                    if (!good) {
-                                        state = 0;
-                                        latch_error(p.err, STREE_ERR_BAD_PATH, b, q, j);
-                                        break;
-                                    }
-                                    pnode[q] = (int16_t)j;
-                                }
                             }
                         }
                     }
                     misc[M_LEN] = len;
                     misc[M_STATE] = state;
-                    int acc = 0;
-                    for (int i = 0; i < T; ++i) {
-                        poff[i] = acc;
-                        for (int w = 0; w < W; ++w) acc += __popc(ancs[i * W + w]);
+                }
+            }
+            __syncthreads();
+            if (new_b) {
+                // Every path position q must hold the depth-q ancestor of the last node.
+                const int len = misc[M_LEN];
+                if (misc[M_STATE] && len > 0) {
+                    const int leaf = __ldg(&p.path[(size_t)b * p.maxlen + len - 1]);
+                    for (int q = tid; q < len; q += kThreads) {
+                        const int j = __ldg(&p.path[(size_t)b * p.maxlen + q]);
+                        const bool good = j >= 0 && j < T && ((ancs[leaf * W + (j >> 5)] >> (j & 31)) & 1u) &&
+                                          __ldg(&p.tree.depth[(size_t)b * T + j]) == q;
+                        if (!good) {
+                            misc[M_STATE] = 0;
+                            latch_error(p.err, STREE_ERR_BAD_PATH, b, q, j);
+                        }
+                        pnode[q] = (int16_t)(good ? j : 0);
                     }
-                    poff[T] = acc;
-                    misc[M_TOTAL] = acc;
-                    misc[M_INSMEM] = acc <= p.pair_cap;
+                }
+                // Pair offsets: exclusive prefix sum of the ancestor counts (T <= 128).
+                int cnt = 0;
+                if (tid < T)
+                    for (int w = 0; w < W; ++w) cnt += __popc(ancs[tid * W + w]);
+                int incl = cnt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                if (lane == 31) misc[M_WSUM + warp] = incl;
+                __syncthreads();
+                int add = 0;
+                for (int w = 0; w < warp; ++w) add += misc[M_WSUM + w];
+                if (tid < T) poff[tid + 1] = add + incl;
+                if (tid == 0) {
+                    poff[0] = 0;
+                    int total = 0;
+                    for (int w = 0; w < kThreads / 32; ++w) total += misc[M_WSUM + w];
+                    misc[M_TOTAL] = total;
+                    misc[M_INSMEM] = total <= p.pair_cap;
                 }
                 cur_b = b;
             }
-            // C operand: rows i < T_pad, fp32 in the 128-byte swizzled K-major layout.
-            for (int q = tid; q < p.T_pad * 32; q += kThreads) {
-                const int i = q >> 5, c = q & 31;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < T) {
-                    const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p.C + (((size_t)b * T + i) * G + g) * kDstate + c * 4));
-                    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
-                    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
-                    v = make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
-                }
-                const int kb = c >> 3, ch = c & 7;
-                *reinterpret_cast<float4 *>(cs + kb * p.T_pad * 128 + i * 128 + ((ch ^ (i & 7)) << 4)) = v;
-            }
             __syncthreads();
+            {
+                const int len = min(misc[M_LEN], kPathRows);
+                if (misc[M_STATE])
+                    for (int q = tid; q < len * 16; q += kThreads)
+                        reinterpret_cast<uint4 *>(Bp)[q] =
+                            __ldg(reinterpret_cast<const uint4 *>(Bseq + (size_t)pnode[q >> 4] * brow) + (q & 15));
+            }
             if (misc[M_INSMEM]) {
                 const int total = misc[M_TOTAL];
-                const float *cbg = p.cb + ((size_t)b * G + g) * T * T;
                 for (int q = tid; q < total; q += kThreads) {
                     int lo = 0, hi = T;                   // poff[lo] <= q < poff[hi]
                     while (hi - lo > 1) {
@@ -225,7 +350,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     const int j = nth_set_bit(ancs + lo * W, W, q - poff[lo]);
                     pj[q] = (uint8_t)j;
-                    pcb[q] = __ldg(&cbg[(size_t)lo * T + j]);
+                    pcb[q] = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, lo);
                 }
             }
             ptx::fence_proxy_async_smem();
@@ -234,8 +359,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         }
 
         const int nt = next_valid(t + 1);
+        uint8_t *h0t = h0s + stage * h0_stage_bytes;
+        uint8_t *xt = xs + stage * p.x_stage;
 
-        // ---------------------------------------------------- MMA + prefetch (one thread)
+        // ---------------------------------------------------- root MMA + prefetch (one thread)
         if (tid == 0) {
             if (!ptx::mbar_wait(bar_full0 + 8u * stage, (k >> 1) & 1)) {
                 latch_error(p.err, STREE_ERR_TIMEOUT, b, r0, 1);
@@ -243,16 +370,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             } else {
                 pending_load = false;
                 ptx::tc_fence_after();
-                const uint32_t a0 = ptx::smem_u32(h0s + stage * h0_stage_bytes);
+                const uint32_t a0 = ptx::smem_u32(h0t);
                 const uint32_t b0 = ptx::smem_u32(cs);
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         ptx::mma_tf32(tmem, ptx::desc_kmajor_sw128(a0 + kb * RB * 128 + kk * 32),
-                                      ptx::desc_kmajor_sw128(b0 + kb * p.T_pad * 128 + kk * 32), idesc,
+                                      ptx::desc_kmajor_sw128(b0 + kb * T_pad * 128 + kk * 32), idesc_root,
                                       (kb | kk) != 0);
-                ptx::mma_commit(bar_mma);
                 if (nt < end) {
                     ptx::bulk_wait_read_all();            // tile k-1's stores have left the other stage
                     issue_load(nt, stage ^ 1);
@@ -260,14 +386,20 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 }
             }
         }
+        __syncthreads();
+        if (misc[M_ABORT]) break;
 
         // ---------------------------------------------------- per-tile coefficients
         const int hpt = p.hpt;
         const int len = misc[M_LEN];
         const bool commit = p.do_commit && misc[M_STATE];
-        for (int q = tid; q < hpt * T; q += kThreads) {
-            const int hh = q / T, i = q - hh * T;
-            dts[q] = bf2f(p.dt[((size_t)b * T + i) * H + hfirst + hh]);
+        {
+            const __nv_bfloat16 *dtt = reinterpret_cast<const __nv_bfloat16 *>(xt + p.x_dt);
+            const int hoff = hfirst - (hfirst & ~7);
+            for (int q = tid; q < hpt * T; q += kThreads) {
+                const int hh = q / T, i = q - hh * T;
+                dts[q] = bf2f(dtt[i * p.dt_box + hoff + hh]);
+            }
         }
         __syncthreads();
         for (int q = tid; q < hpt * T; q += kThreads) {
@@ -286,6 +418,38 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             eLs[q] = expf(L);
         }
         __syncthreads();
+        // Masked decay matrix of every head of the tile (bf16, K-major swizzled):
+        // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i.
+        {
+            const int total = misc[M_TOTAL];
+            const bool insmem = misc[M_INSMEM] != 0;
+            for (int q = tid; q < hpt * total; q += kThreads) {
+                const int hh = q / total, qq = q - hh * total;
+                int i, j;
+                float cbv;
+                if (insmem) {
+                    int lo = 0, hi = T;
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if (poff[mid] <= qq) lo = mid; else hi = mid;
+                    }
+                    i = lo;
+                    j = pj[qq];
+                    cbv = pcb[qq];
+                } else {
+                    int lo = 0, hi = T;
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if (poff[mid] <= qq) lo = mid; else hi = mid;
+                    }
+                    i = lo;
+                    j = nth_set_bit(ancs + i * W, W, qq - poff[i]);
+                    cbv = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i);
+                }
+                const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * cbv * dts[hh * T + j];
+                *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) = __float2bfloat16_rn(m);
+            }
+        }
         if (commit) {
             const int leaf = len > 0 ? pnode[len - 1] : 0;
             for (int q = tid; q < hpt * len; q += kThreads) {
@@ -295,92 +459,67 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             if (tid < hpt) alpha[tid] = len > 0 ? eLs[tid * T + leaf] : 1.f;
         }
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
 
-        // ---------------------------------------------------- wait for the MMA
-        if (!misc[M_ABORT]) {
-            if (!ptx::mbar_wait(bar_mma, k & 1)) {
-                latch_error(p.err, STREE_ERR_TIMEOUT, b, r0, 2);
-                misc[M_ABORT] = 1;
+        // ---------------------------------------------------- tree MMAs (one thread)
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            const uint32_t xa = ptx::smem_u32(xt);
+            for (int hh = 0; hh < hpt; ++hh) {
+                const uint32_t mb = ptx::smem_u32(mh + hh * p.mh_head);
+                const uint32_t dcol = tmem + (uint32_t)(T_pad * (1 + hh));
+                for (int ks = 0; ks < T_pad / 16; ++ks)
+                    ptx::mma_f16(dcol, ptx::desc_mnmajor_sw128(xa + ks * 2048, xbs, 1024),
+                                 ptx::desc_kmajor_sw128(mb + (ks >> 2) * T_pad * 128 + (ks & 3) * 32), idesc_tree,
+                                 ks != 0);
             }
+            ptx::mma_commit(bar_mma);
+        }
+
+        // ---------------------------------------------------- wait for the MMAs
+        if (!ptx::mbar_wait(bar_mma, k & 1)) {
+            latch_error(p.err, STREE_ERR_TIMEOUT, b, r0, 2);
+            misc[M_ABORT] = 1;
         }
         __syncthreads();
         if (misc[M_ABORT]) break;
         ptx::tc_fence_after();
 
-        uint8_t *h0t = h0s + stage * h0_stage_bytes;
-        __nv_bfloat16 *xt = reinterpret_cast<__nv_bfloat16 *>(xs + stage * p.x_stage);
-
         // ---------------------------------------------------- commit, in place over h0
         if (commit) {
-            const int row = tid % RB, seg = tid / RB;     // RB columns per thread
+            const int tpr = kThreads / RB;                 // threads per row
+            const int row = tid % RB, part = tid / RB;
             const int hh = (r0 + row) / P - hfirst;
-            const float al = alpha[hh];
-            const float *wh = wts + hh * T;
-            for (int c4 = 0; c4 < RB / 4; ++c4) {
-                const int n = seg * RB + c4 * 4;
-                const int kb = n >> 5, ch = (n & 31) >> 2;
-                float4 *ptr = reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
-                float4 v = *ptr;
-                v.x *= al; v.y *= al; v.z *= al; v.w *= al;
-                for (int q = 0; q < len; ++q) {
-                    const int j = pnode[q];
-                    const float coef = wh[q] * bf2f(xt[j * RB + row]);
-                    const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p.B + (((size_t)b * T + j) * G + g) * kDstate + n));
-                    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
-                    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
-                    v.x = fmaf(coef, __low2float(lo), v.x);
-                    v.y = fmaf(coef, __high2float(lo), v.y);
-                    v.z = fmaf(coef, __low2float(hi), v.z);
-                    v.w = fmaf(coef, __high2float(hi), v.w);
-                }
-                *ptr = v;
-            }
+            if (tpr == 2)
+                commit_rows<64>(h0t, xt, xbs, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 64);
+            else
+                commit_rows<32>(h0t, xt, xbs, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 32);
         }
         __syncthreads();                                   // x rows of the path are read
 
         // ---------------------------------------------------- y, in place over x
-        if (warp < RB / 32) {
-            const int row = warp * 32 + lane;
-            const int hh = (r0 + row) / P - hfirst;       // same for the whole warp (P >= 32)
-            const float Dh = __ldg(&p.D[hfirst + hh]);
-            const float *Lh = Ls + hh * T, *eLh = eLs + hh * T, *dth = dts + hh * T;
-            const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-            const bool insmem = misc[M_INSMEM] != 0;
-            const float *cbg = p.cb + ((size_t)b * G + g) * T * T;
-            __nv_bfloat16 *xc = xt + row;
-            for (int c0 = ((T - 1) >> 4) << 4; c0 >= 0; c0 -= 16) {
-                float v[16];
-                ptx::tmem_ld16(tl + (uint32_t)c0, v);
+        {
+            const int quad = warp & 3, half = warp >> 2;
+            if (quad * 32 < RB) {
+                const int row = quad * 32 + lane;
+                const int hh = (r0 + row) / P - hfirst;   // same for the whole warp (P >= 32)
+                const float Dh = __ldg(&p.D[hfirst + hh]);
+                const float *eLh = eLs + hh * T;
+                const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+                const uint32_t ty = tl + (uint32_t)(T_pad * (1 + hh));
+                for (int c0 = half * 16; c0 < T; c0 += 32) {
+                    float R[16], Y[16];
+                    ptx::tmem_ld16(tl + (uint32_t)c0, R);
+                    ptx::tmem_ld16(ty + (uint32_t)c0, Y);
 #pragma unroll
-                for (int u = 15; u >= 0; --u) {
-                    const int i = c0 + u;
-                    if (i < T) {
-                        const float Li = Lh[i];
-                        float tree = 0.f;
-                        const int q0 = poff[i], cnt = poff[i + 1] - q0;
-                        for (int base = 0; base < cnt; base += 32) {
-                            int jl = 0;
-                            float ml = 0.f;
-                            if (base + lane < cnt) {
-                                float cbv;
-                                if (insmem) {
-                                    jl = pj[q0 + base + lane];
-                                    cbv = pcb[q0 + base + lane];
-                                } else {
-                                    jl = nth_set_bit(ancs + i * W, W, base + lane);
-                                    cbv = __ldg(&cbg[(size_t)i * T + jl]);
-                                }
-                                ml = expf(Li - Lh[jl]) * cbv * dth[jl];
-                            }
-                            const int nn = min(32, cnt - base);
-                            for (int s = 0; s < nn; ++s) {
-                                const float ms = __shfl_sync(0xffffffffu, ml, s);
-                                const int js = __shfl_sync(0xffffffffu, jl, s);
-                                tree = fmaf(ms, bf2f(xc[js * RB]), tree);
-                            }
+                    for (int u = 0; u < 16; ++u) {
+                        const int i = c0 + u;
+                        if (i < T) {
+                            __nv_bfloat16 *xe = reinterpret_cast<__nv_bfloat16 *>(xt + mn_off(i, row, xbs));
+                            const float yv = fmaf(eLh[i], R[u], fmaf(Dh, bf2f(*xe), Y[u]));
+                            *xe = __float2bfloat16_rn(yv);
                         }
-                        const float yv = eLh[i] * v[u] + tree + Dh * bf2f(xc[i * RB]);
-                        xc[i * RB] = __float2bfloat16_rn(yv);
                     }
                 }
             }
@@ -391,7 +530,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
 
         // ---------------------------------------------------- stores (one thread)
         if (tid == 0) {
-            ptx::tma_store_2d(&tm_y, r0, b * T, ptx::smem_u32(xt));
+            const uint32_t xsrc = ptx::smem_u32(xt);
+            for (int nb = 0; nb < p.NB; ++nb)
+                ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
             if (commit) {
                 const uint32_t src = ptx::smem_u32(h0t);
                 for (int kb = 0; kb < 4; ++kb)
@@ -460,30 +601,39 @@ bool layout(const ScanArgs &a, int RB, TcParams &p, size_t &smem)
 {
     const int T = a.T, T_pad = (T + 15) / 16 * 16, W = (T + 31) / 32;
     const int hpt = a.P >= RB ? 1 : RB / a.P;
+    const int NB = RB / 64, KA = (T_pad + 63) / 64;
+    p.dt_box = a.H < kDtBox ? a.H : kDtBox;
     uint32_t off = 2u * RB * 512u;                            // h0 stages
     p.off_x = off;
-    p.x_stage = round_up((uint32_t)T * RB * 2u, 1024u);
-    uint32_t xreg = 2u * p.x_stage;
-    const uint32_t spill = (uint32_t)(128 - RB) * 128u;      // MMA rows past the last h0 stage
-    if (xreg < spill) xreg = spill;
-    off = round_up(off + xreg, 1024u);
-    p.off_c = off;
-    off += (uint32_t)T_pad * 512u;
-    p.off_anc = off;   off = round_up(off + (uint32_t)T * W * 4u, 16u);
-    p.off_poff = off;  off = round_up(off + (uint32_t)(T + 1) * 4u, 16u);
-    p.off_dts = off;   off = round_up(off + (uint32_t)hpt * T * 4u, 16u);
-    p.off_L = off;     off = round_up(off + (uint32_t)hpt * T * 4u, 16u);
-    p.off_eL = off;    off = round_up(off + (uint32_t)hpt * T * 4u, 16u);
-    p.off_w = off;     off = round_up(off + (uint32_t)hpt * T * 4u, 16u);
-    p.off_alpha = off; off = round_up(off + (uint32_t)hpt * 4u, 16u);
-    p.off_pnode = off; off = round_up(off + (uint32_t)T * 2u, 16u);
-    p.off_bar = off;   off = round_up(off + 3u * 8u, 16u);
-    p.off_misc = off;  off = round_up(off + kMiscWords * 4u, 16u);
-    p.off_pcb = off;
-    const size_t fixed = (size_t)off + 1024;                  // + alignment slack of the dynamic base
-    if (fixed + 5 * 64 > kSmemLimit) return false;
+    p.x_dt = (uint32_t)NB * T_pad * 128u;
+    p.x_stage = round_up(p.x_dt + (uint32_t)T * p.dt_box * 2u, 1024u);
+    off += 2u * p.x_stage;
+    // MMA rows past the tile (h0 rows >= RB, the second x block when RB = 64)
+    // read whatever follows; keep that inside the allocation.
+    const uint32_t spill = (uint32_t)(128 - RB) * 128u > (uint32_t)T_pad * 128u ? (uint32_t)(128 - RB) * 128u
+                                                                               : (uint32_t)T_pad * 128u;
+    p.off_c = round_up(off, 1024u);
+    off = p.off_c + (uint32_t)T_pad * 512u;
+    if (off < p.off_c + spill) off = p.off_c + spill;
+    p.off_mh = round_up(off, 1024u);
+    p.mh_head = (uint32_t)KA * T_pad * 128u;
+    off = p.off_mh + (uint32_t)hpt * p.mh_head;
+    p.off_bp = round_up(off, 16u);     off = p.off_bp + (uint32_t)kPathRows * kDstate * 2u;
+    p.off_anc = round_up(off, 16u);    off = p.off_anc + (uint32_t)T * W * 4u;
+    p.off_poff = round_up(off, 16u);   off = p.off_poff + (uint32_t)(T + 1) * 4u;
+    p.off_dts = round_up(off, 16u);    off = p.off_dts + (uint32_t)hpt * T * 4u;
+    p.off_L = round_up(off, 16u);      off = p.off_L + (uint32_t)hpt * T * 4u;
+    p.off_eL = round_up(off, 16u);     off = p.off_eL + (uint32_t)hpt * T * 4u;
+    p.off_w = round_up(off, 16u);      off = p.off_w + (uint32_t)hpt * T * 4u;
+    p.off_alpha = round_up(off, 16u);  off = p.off_alpha + (uint32_t)hpt * 4u;
+    p.off_pnode = round_up(off, 16u);  off = p.off_pnode + (uint32_t)T * 2u;
+    p.off_bar = round_up(off, 16u);    off = p.off_bar + 3u * 8u;
+    p.off_misc = round_up(off, 16u);   off = p.off_misc + kMiscWords * 4u;
+    p.off_pcb = round_up(off, 16u);
+    const size_t fixed = (size_t)p.off_pcb + 1024;            // + alignment slack of the dynamic base
+    if (fixed + 5 * 64 + 16 > kSmemLimit) return false;
     const int all_pairs = T * (T + 1) / 2;
-    int cap = (int)((kSmemLimit - fixed) / 5);
+    int cap = (int)((kSmemLimit - fixed - 16) / 5);
     if (cap > all_pairs) cap = all_pairs;
     p.pair_cap = cap;
     p.off_pj = round_up(p.off_pcb + (uint32_t)cap * 4u, 16u);
@@ -492,10 +642,13 @@ bool layout(const ScanArgs &a, int RB, TcParams &p, size_t &smem)
     if (smem > kSmemLimit) return false;
     p.T = T;
     p.T_pad = T_pad;
+    p.KA = KA;
     p.RB = RB;
+    p.NB = NB;
     p.hpt = hpt;
     uint32_t cols = 32;
-    while (cols < (uint32_t)T_pad) cols <<= 1;
+    while (cols < (uint32_t)((1 + hpt) * T_pad)) cols <<= 1;
+    if (cols > 512) return false;
     p.tmem_cols = cols;
     return true;
 }
@@ -510,17 +663,19 @@ bool rb_valid(const ScanArgs &a, int RB)
 
 bool plan(const ScanArgs &a, TcPlan &pl)
 {
-    if (a.dtype != STREE_BF16 || a.N != kDstate || a.T > kMaxTcNodes || a.P % 32 != 0) return false;
+    if (a.dtype != STREE_BF16 || a.N != kDstate || a.T > kMaxTcNodes || a.P % 32 != 0 || a.H % 8 != 0) return false;
     if (a.batch <= 0 || a.H % a.G != 0) return false;
     if (!encode_fn()) return false;
     const int sms = num_sms();
     int chosen = -1;
     TcParams best{};
     size_t best_smem = 0;
-    for (int RB : {128, 64, 32}) {
+    for (int RB : {128, 64}) {
         TcParams p{};
         size_t smem = 0;
         if (!rb_valid(a, RB) || !layout(a, RB, p, smem)) continue;
+        // Room for the ancestor pairs of typical trees (about 4 per node).
+        if (p.pair_cap < 4 * a.T && p.pair_cap < a.T * (a.T + 1) / 2 && RB > 64) continue;
         const long long ntiles = (long long)a.batch * (a.H * a.P / RB);
         if (ntiles > 0x7fffffff) continue;
         chosen = RB;
@@ -552,7 +707,6 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     TcPlan pl;
     if (!plan(a, pl)) return cudaErrorNotSupported;
     TcParams p = pl.p;
-    p.dt = static_cast<const __nv_bfloat16 *>(a.dt);
     p.B = static_cast<const __nv_bfloat16 *>(a.B);
     p.C = static_cast<const __nv_bfloat16 *>(a.C);
     p.A = a.A;
@@ -561,13 +715,12 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     p.path_len = a.path_len;
     p.maxlen = a.maxlen;
     p.do_commit = a.path != nullptr && a.h_new != nullptr;
-    p.cb = a.cb;
     p.tree = a.tree;
     p.err = a.err;
 
     EncodeTiledFn enc = encode_fn();
     const int HP = a.H * a.P;
-    CUtensorMap m_h0, m_hn, m_x, m_y;
+    CUtensorMap m_h0, m_hn, m_x, m_y, m_dt;
     {
         cuuint64_t dims[2] = {(cuuint64_t)kDstate, (cuuint64_t)a.batch * HP};
         cuuint64_t strides[1] = {(cuuint64_t)kDstate * 4};
@@ -586,19 +739,30 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     {
         cuuint64_t dims[2] = {(cuuint64_t)HP, (cuuint64_t)a.batch * a.T};
         cuuint64_t strides[1] = {(cuuint64_t)HP * 2};
-        cuuint32_t box[2] = {(cuuint32_t)p.RB, (cuuint32_t)a.T};
+        cuuint32_t box[2] = {64, (cuuint32_t)a.T};
         cuuint32_t es[2] = {1, 1};
         if (enc(&m_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.x), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
         if (enc(&m_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.y, dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)a.H, (cuuint64_t)a.batch * a.T};
+        cuuint64_t strides[1] = {(cuuint64_t)a.H * 2};
+        cuuint32_t box[2] = {(cuuint32_t)p.dt_box, (cuuint32_t)a.T};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&m_dt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.dt), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
     if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int per_sm = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_tc_kernel, kThreads, pl.smem) != cudaSuccess ||
         per_sm < 1)
@@ -608,7 +772,7 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     if (per_sm > tmem_fit) per_sm = tmem_fit;
     long long grid = (long long)num_sms() * per_sm;
     if (grid > p.ntiles) grid = p.ntiles;
-    scan_tc_kernel<<<(unsigned)grid, kThreads, pl.smem, s>>>(m_h0, m_hn, m_x, m_y, p);
+    scan_tc_kernel<<<(unsigned)grid, kThreads, pl.smem, s>>>(m_h0, m_hn, m_x, m_y, m_dt, p);
     return cudaGetLastError();
 }
 

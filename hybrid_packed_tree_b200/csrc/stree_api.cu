@@ -118,6 +118,8 @@ stree_status run_scan(stree_ctx *c, ScanArgs &a, cudaStream_t s)
     } else if (c->kernel == STREE_KERNEL_AUTO) {
         use_tc = tc_supported(a);
     }
+    ++c->launches;
+    if (use_tc) return cuda_status(launch_scan_tc(a, s));     // computes C.B pairs itself
     stree_status st = ensure(&c->cb, &c->cap_cb, (size_t)a.batch * a.G * a.T * a.T);
     if (st != STREE_OK) return st;
     a.cb = c->cb;
@@ -125,8 +127,6 @@ stree_status run_scan(stree_ctx *c, ScanArgs &a, cudaStream_t s)
         ++c->launches;
         if ((st = cuda_status(launch_cb_pairs(a, s))) != STREE_OK) return st;
     }
-    ++c->launches;
-    if (use_tc) return cuda_status(launch_scan_tc(a, s));
     return cuda_status(launch_scan_simt(a, s));
 }
 

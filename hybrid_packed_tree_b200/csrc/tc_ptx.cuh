@@ -167,6 +167,41 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr)
            | ((uint64_t)2 << 61);                   // 128-byte swizzle
 }
 
+// Shared-memory matrix descriptor: MN-major operand in the canonical 128-byte
+// swizzled layout: 64 bf16 of the M/N dimension per 128-byte row, one row per K
+// index, 8-row groups `sbo` bytes apart along K, 64-wide M/N blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4)
+           | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16)
+           | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32)
+           | ((uint64_t)1 << 46)
+           | ((uint64_t)2 << 61);
+}
+
+// D[tmem] (+)= A * B^T, kind::f16 (bf16 operands here), one CTA.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A (MN-major) and bf16 B (K-major).
+__host__ __device__ constexpr uint32_t idesc_bf16_amn(int M, int N)
+{
+    return (1u << 4)                   // D format: f32
+           | (1u << 7)                 // A format: bf16
+           | (1u << 10)                // B format: bf16
+           | (1u << 15)                // A is MN-major
+           | ((uint32_t)(N >> 3) << 17)
+           | ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor, kind::tf32: fp32 accumulate, tf32 A and B, both K-major.
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N)
 {
