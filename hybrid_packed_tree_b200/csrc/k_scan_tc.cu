@@ -5,24 +5,31 @@
 // one scan over the packed tree with the accumulated transition A_tree = L.logA,
 // and the accepted path's state is rebuilt by activation replay:
 //   L_i   = A_h * sum_{j in anc(i)} dt_j
-//   y_i   = exp(L_i) (h0 . C_i) + sum_{j in anc(i)} exp(L_i - L_j) cb_ij dt_j x_j + D_h x_i
+//   y_i   = exp(L_i) (h0 . C_i) + sum_{j in anc(i)} exp(L_i - L_j) (C_i . B_j) dt_j x_j + D_h x_i
 //   h_new = exp(L_leaf) h0 + sum_{j on path} exp(L_leaf - L_j) dt_j x_j (outer) B_j
 //
-// Design (B200): the state h0 [b, H*P, N] is streamed through the SMs in tiles of
-// RB rows of the flattened (head, headdim) axis.  Per tile:
-//   * TMA brings the fp32 h0 tile (128-byte swizzled, 4 boxes of 32 columns) and
-//     the bf16 x tile [T nodes x RB] into a double-buffered stage;
-//   * one thread issues tcgen05.mma kind::tf32 (M = 128, N = T_pad, K = 128):
-//     R[row, i] = h0[row, :] . C_i[:] into tensor memory -- the root term, the
-//     only dense contraction of the path (C is staged once per sequence/group);
-//   * the commit (fp32 FMA, exact h0) is written in place over the h0 tile and
-//     the outputs y in place over the x tile; TMA stores both back;
-//   * the sparse tree term runs on the CUDA cores over the ancestor pairs only
-//     (lanes of a warp share a head: each lane builds one pair's decayed weight
-//     and the warp broadcasts them), so exp never sees a positive argument.
-// The load of tile k+1 and the stores of tile k-1 overlap the work on tile k.
-// Only the tf32 rounding of h0 inside the root-term MMA departs from fp32
-// arithmetic; it is below the bf16 rounding of the output y.
+// Design (B200).  The state h0 [b, H*P, N=128] streams through the SMs in tiles
+// of RB rows of the flattened (head, headdim) axis; a persistent CTA walks a
+// contiguous range of tiles with warp-specialised roles joined by mbarriers:
+//   * producer warp: TMA loads of the fp32 h0 tile (128-byte swizzled, 4 boxes
+//     of 32 columns), the bf16 x tile (64-column swizzled boxes) and the dt box
+//     into a 2-stage ring;
+//   * MMA warp (one thread): the root term R[row, i] = h0[row, :] . C_i as
+//     tcgen05.mma kind::tf32 (M = 128, N = T_pad, K = 128) and the tree term
+//     Y[row, i] = sum_j x[j, row] M_h[i, j] as kind::f16 with x as an MN-major
+//     operand straight from the stage, into a 2-deep tensor-memory ring;
+//   * prep warps: per tile and head the tree cumsum L, exp(L) and the masked
+//     decay matrix M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j over ancestor
+//     pairs only (bf16, K-major swizzled), plus the commit weights;
+//   * epilogue warps: the commit in exact fp32 FMA, written in place over the
+//     h0 tile, then y = exp(L_i) R + Y + D x in place over the x tile, then TMA
+//     stores of both and the release of the stage.
+// C (fp32 operand of the root MMA), the ancestor pairs' C.B and the accepted
+// path's rows of B are staged once per (sequence, group).  Roles only block on
+// bounded mbarrier waits; a timeout latches STREE_ERR_TIMEOUT and the CTA runs
+// to its end without further work.  Precision: the root term rounds h0 to tf32
+// and the masked decay matrix to bf16 inside the MMAs (fp32 accumulation); the
+// commit and every other step are fp32.
 #include <cuda.h>
 
 #include <mutex>
@@ -33,14 +40,21 @@
 namespace stree {
 namespace {
 
-constexpr int kThreads = 256;
 constexpr int kDstate = 128;               // dstate of the tensor-core path
 constexpr int kMaxTcNodes = 128;           // T_pad <= 128 (TMEM columns, smem)
 constexpr int kDtBox = 16;                 // heads per dt box (32 bytes of bf16)
-constexpr int kPathRows = 16;              // accepted-path rows of B staged in smem
+constexpr int kPathRows = 8;               // accepted-path rows of B staged in smem (fp32)
 constexpr size_t kSmemLimit = 232448;      // 227 KB opt-in dynamic shared memory
 
-enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_WSUM = 8, kMiscWords = 16 };
+constexpr int kProducerWarp = 0, kMmaWarp = 1, kPrepWarp0 = 2, kPrepWarps = 2, kEpiWarp0 = 4, kEpiWarps = 8;
+constexpr int kWarps = kEpiWarp0 + kEpiWarps;
+constexpr int kThreads = kWarps * 32;
+constexpr int kPrepThreads = kPrepWarps * 32, kEpiThreads = kEpiWarps * 32;
+constexpr int kBarEpi = 1, kBarPrep = 2;   // named barriers (0 is __syncthreads)
+
+enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_WSUM = 8, kMiscWords = 8 + kWarps };
+enum Bars { B_FULL = 0, B_EMPTY = 2, B_ACCF = 4, B_ACCE = 6, B_MHF = 8, B_MHE = 9, B_COEFF = 10, B_COEFE = 12,
+            kNumBars = 14 };
 
 struct TcParams {
     const __nv_bfloat16 *__restrict__ B;
@@ -51,10 +65,10 @@ struct TcParams {
     const int32_t *__restrict__ path_len;
     TreeView tree;
     int32_t *err;
-    int T, T_pad, KA, H, P, G, RB, NB, tps, ntiles, maxlen, do_commit, hpt, pair_cap, dt_box;
+    int T, T_pad, KA, H, P, G, RB, NB, tps, ntiles, maxlen, do_commit, hpt, pair_cap, dt_box, acc_cols;
     uint32_t tmem_cols;
-    uint32_t off_x, x_dt, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_dts, off_L, off_eL,
-        off_w, off_alpha, off_pnode, off_bar, off_misc, off_pcb, off_pj;
+    uint32_t off_x, x_dt, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_coef, coef_slot,
+        off_pnode, off_bar, off_misc, off_pcb, off_pj;
 };
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -79,6 +93,17 @@ __device__ __forceinline__ int nth_set_bit(const uint32_t *row, int W, int n)
     return -1;
 }
 
+// Index i with poff[i] <= q < poff[i+1] (poff non-decreasing, poff[0] = 0).
+__device__ __forceinline__ int pair_row(const int32_t *poff, int T, int q)
+{
+    int lo = 0, hi = T;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (poff[mid] <= q) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
 // C_i . B_j: C from the staged fp32 MMA operand (swizzled), B_j from global memory.
 __device__ __forceinline__ float dot_cb(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i)
 {
@@ -98,14 +123,6 @@ __device__ __forceinline__ float dot_cb(const uint8_t *cs, int T_pad, const __nv
     return acc;
 }
 
-// Byte offset of bf16 element (k row, m column) in an MN-major 128-byte swizzled
-// block stack: 64 columns per block, blocks `bstride` bytes apart.
-__device__ __forceinline__ uint32_t mn_off(int krow, int m, uint32_t bstride)
-{
-    return (uint32_t)(m >> 6) * bstride + (uint32_t)krow * 128u +
-           ((uint32_t)(((m & 63) >> 3) ^ (krow & 7)) << 4) + (uint32_t)(m & 7) * 2u;
-}
-
 // Byte offset of bf16 element (row, k) in a K-major 128-byte swizzled operand of
 // `rows` rows: 64 K-columns per atom, atoms rows*128 bytes apart.
 __device__ __forceinline__ uint32_t k_off(int row, int kcol, int rows)
@@ -114,11 +131,24 @@ __device__ __forceinline__ uint32_t k_off(int row, int kcol, int rows)
            ((uint32_t)(((kcol & 63) >> 3) ^ (row & 7)) << 4) + (uint32_t)(kcol & 7) * 2u;
 }
 
+// Column `m` of an MN-major 128-byte swizzled bf16 stack (64 columns per block,
+// blocks xbs bytes apart): element (k, m) sits at base + k*128 + ((chunk ^ (k&7)) << 4).
+struct MnCol {
+    uint32_t base, chunk;
+    __device__ __forceinline__ MnCol(int m, uint32_t xbs)
+        : base((uint32_t)(m >> 6) * xbs + (uint32_t)(m & 7) * 2u), chunk((uint32_t)((m & 63) >> 3)) {}
+    __device__ __forceinline__ uint32_t at(int k) const
+    {
+        return base + (uint32_t)k * 128u + ((chunk ^ (uint32_t)(k & 7)) << 4);
+    }
+};
+
 // Commit of one tile row segment: h_new = alpha h0 + sum_q coef_q B[pnode_q] (fp32).
-// The first kPathRows path rows of B come from shared memory, later ones from global.
+// The first kPathRows path rows of B come from shared memory (fp32), later ones
+// from global memory.
 template <int CPT>
-__device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, uint32_t xbs, const __nv_bfloat16 *Bp,
-                                            const __nv_bfloat16 *Bseq, size_t brow_stride, const int16_t *pnode,
+__device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, const MnCol &xc, const float *Bp,
+                                            const __nv_bfloat16 *Bseq, size_t brow, const int16_t *pnode,
                                             const float *wh, float al, int len, int RB, int row, int c_lo)
 {
     float acc[CPT];
@@ -126,17 +156,28 @@ __device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, uin
     for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
     for (int q = 0; q < len; ++q) {
         const int j = pnode[q];
-        const float coef = wh[q] * bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + mn_off(j, row, xbs)));
-        const uint2 *src = q < kPathRows ? reinterpret_cast<const uint2 *>(Bp + q * kDstate + c_lo)
-                                         : reinterpret_cast<const uint2 *>(Bseq + (size_t)j * brow_stride + c_lo);
+        const float coef = wh[q] * bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
+        if (q < kPathRows) {
+            const float4 *src = reinterpret_cast<const float4 *>(Bp + q * kDstate + c_lo);
 #pragma unroll
-        for (int c = 0; c < CPT / 4; ++c) {
-            float b0, b1, b2, b3;
-            unpack4(src[c], b0, b1, b2, b3);
-            acc[4 * c + 0] = fmaf(coef, b0, acc[4 * c + 0]);
-            acc[4 * c + 1] = fmaf(coef, b1, acc[4 * c + 1]);
-            acc[4 * c + 2] = fmaf(coef, b2, acc[4 * c + 2]);
-            acc[4 * c + 3] = fmaf(coef, b3, acc[4 * c + 3]);
+            for (int c = 0; c < CPT / 4; ++c) {
+                const float4 bv = src[c];
+                acc[4 * c + 0] = fmaf(coef, bv.x, acc[4 * c + 0]);
+                acc[4 * c + 1] = fmaf(coef, bv.y, acc[4 * c + 1]);
+                acc[4 * c + 2] = fmaf(coef, bv.z, acc[4 * c + 2]);
+                acc[4 * c + 3] = fmaf(coef, bv.w, acc[4 * c + 3]);
+            }
+        } else {
+            const uint2 *src = reinterpret_cast<const uint2 *>(Bseq + (size_t)j * brow + c_lo);
+#pragma unroll
+            for (int c = 0; c < CPT / 4; ++c) {
+                float b0, b1, b2, b3;
+                unpack4(__ldg(src + c), b0, b1, b2, b3);
+                acc[4 * c + 0] = fmaf(coef, b0, acc[4 * c + 0]);
+                acc[4 * c + 1] = fmaf(coef, b1, acc[4 * c + 1]);
+                acc[4 * c + 2] = fmaf(coef, b2, acc[4 * c + 2]);
+                acc[4 * c + 3] = fmaf(coef, b3, acc[4 * c + 3]);
+            }
         }
     }
 #pragma unroll
@@ -153,6 +194,16 @@ __device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, uin
     }
 }
 
+__device__ __forceinline__ void named_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant__ CUtensorMap tm_hn,
                const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
@@ -162,33 +213,29 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = p.T, T_pad = p.T_pad, RB = p.RB, P = p.P, H = p.H, G = p.G, W = p.tree.W, HP = H * P;
-    const int hpg = H / G;
+    const int hpg = H / G, hpt = p.hpt;
     const uint32_t xbs = (uint32_t)T_pad * 128u;                      // x: bytes per 64-column block
 
     uint8_t *h0s = smem;                                              // 2 x [4 atoms][RB rows][128 B] fp32
     uint8_t *xs = smem + p.off_x;                                     // 2 x {NB x [T_pad rows][128 B] x, dt}
     uint8_t *cs = smem + p.off_c;                                     // [4 atoms][T_pad rows][128 B] fp32
     uint8_t *mh = smem + p.off_mh;                                    // hpt x [KA atoms][T_pad rows][128 B] bf16
-    __nv_bfloat16 *Bp = reinterpret_cast<__nv_bfloat16 *>(smem + p.off_bp);  // [kPathRows][128]
+    float *Bp = reinterpret_cast<float *>(smem + p.off_bp);           // [kPathRows][128] fp32
     uint32_t *ancs = reinterpret_cast<uint32_t *>(smem + p.off_anc);  // [T][W]
     int32_t *poff = reinterpret_cast<int32_t *>(smem + p.off_poff);   // [T+1]
-    float *dts = reinterpret_cast<float *>(smem + p.off_dts);         // [hpt][T]
-    float *Ls = reinterpret_cast<float *>(smem + p.off_L);            // [hpt][T]
-    float *eLs = reinterpret_cast<float *>(smem + p.off_eL);          // [hpt][T]
-    float *wts = reinterpret_cast<float *>(smem + p.off_w);           // [hpt][T]
-    float *alpha = reinterpret_cast<float *>(smem + p.off_alpha);     // [hpt]
     int16_t *pnode = reinterpret_cast<int16_t *>(smem + p.off_pnode); // [T]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.off_bar);  // full[2], mma
-    int32_t *misc = reinterpret_cast<int32_t *>(smem + p.off_misc);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.off_bar);
+    volatile int32_t *misc = reinterpret_cast<volatile int32_t *>(smem + p.off_misc);
     float *pcb = reinterpret_cast<float *>(smem + p.off_pcb);         // [pair_cap]
     uint8_t *pj = smem + p.off_pj;                                    // [pair_cap]
+    // Per-tile coefficients, two slots: dts, L, exp(L), commit weights [hpt][T] each, alpha [hpt].
+    auto coef = [&](int slot, int which) {
+        return reinterpret_cast<float *>(smem + p.off_coef + slot * p.coef_slot) + which * hpt * T;
+    };
+    auto bar = [&](int i) { return ptx::smem_u32(&bars[i]); };
 
-    const uint32_t bar_full0 = ptx::smem_u32(&bars[0]);
-    const uint32_t bar_mma = ptx::smem_u32(&bars[2]);
     const uint32_t h0_stage_bytes = (uint32_t)RB * 512u;
     const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u + (uint32_t)T * p.dt_box * 2u;
-    const uint32_t idesc_root = ptx::idesc_tf32(128, T_pad);
-    const uint32_t idesc_tree = ptx::idesc_bf16_amn(128, T_pad);
 
     if (tid == 0) {
         ptx::prefetch_tensormap(&tm_h0);
@@ -196,18 +243,25 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         ptx::prefetch_tensormap(&tm_dt);
         ptx::prefetch_tensormap(&tm_hn);
         ptx::prefetch_tensormap(&tm_y);
-        ptx::mbar_init(bar_full0, 1);
-        ptx::mbar_init(bar_full0 + 8, 1);
-        ptx::mbar_init(bar_mma, 1);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(bar(B_FULL + s), 1);
+            ptx::mbar_init(bar(B_EMPTY + s), 1);
+            ptx::mbar_init(bar(B_ACCF + s), 1);
+            ptx::mbar_init(bar(B_ACCE + s), kEpiWarps);
+            ptx::mbar_init(bar(B_COEFF + s), kPrepThreads);
+            ptx::mbar_init(bar(B_COEFE + s), kEpiWarps);
+        }
+        ptx::mbar_init(bar(B_MHF), kPrepThreads);
+        ptx::mbar_init(bar(B_MHE), 1);
         ptx::fence_mbar_init();
-        for (int k = 0; k < kMiscWords; ++k) misc[k] = 0;
+        for (int q = 0; q < kMiscWords; ++q) misc[q] = 0;
     }
     // Operand rows the MMAs read past the valid tile (rows >= RB, nodes >= T)
     // must hold finite values: clear the staging regions once.
     for (uint32_t o = tid * 16u; o < p.off_mh; o += kThreads * 16u)
         *reinterpret_cast<float4 *>(smem + o) = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(&misc[M_TMEM]), p.tmem_cols);
+    if (warp == kMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_u32(const_cast<int32_t *>(&misc[M_TMEM])), p.tmem_cols);
         ptx::tmem_relinquish();
     }
     ptx::fence_proxy_async_smem();
@@ -216,44 +270,57 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     ptx::tc_fence_after();
     const uint32_t tmem = static_cast<uint32_t>(misc[M_TMEM]);
 
+    // Bounded wait that turns a timeout into a CTA-wide abort; after an abort
+    // every wait returns false at once and no role does further work.
+    auto wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
+        if (misc[M_ABORT]) return false;
+        if (ptx::mbar_wait(b, parity)) return true;
+        latch_error(p.err, STREE_ERR_TIMEOUT, blockIdx.x, where, (int)parity);
+        misc[M_ABORT] = 1;
+        return false;
+    };
+
     const int start = (int)((long long)blockIdx.x * p.ntiles / gridDim.x);
     const int end = (int)((long long)(blockIdx.x + 1) * p.ntiles / gridDim.x);
-    auto tile_ok = [&](int t) { return __ldg(&p.tree.ok[t / p.tps]) != 0; };
-    auto next_valid = [&](int t) {
-        while (t < end && !tile_ok(t)) ++t;
-        return t;
-    };
-    auto issue_load = [&](int t, int stage) {
+    uint32_t loads_issued = 0;
+
+    auto produce = [&](uint32_t k, int t) {                    // producer warp, lane 0
+        const int s = k & 1;
+        if (k >= 2 && !wait(bar(B_EMPTY + s), ((k >> 1) - 1) & 1, 10)) return;
+        if (misc[M_ABORT]) return;
         const int b = t / p.tps, r0 = (t % p.tps) * RB;
         const int hf8 = (r0 / P) & ~7;
-        const uint32_t bar = bar_full0 + 8u * stage;
-        ptx::mbar_expect_tx(bar, tx_bytes);
-        const uint32_t dst = ptx::smem_u32(h0s + stage * h0_stage_bytes);
-        for (int kb = 0; kb < 4; ++kb)
-            ptx::tma_load_2d(dst + kb * RB * 128, &tm_h0, kb * 32, b * HP + r0, bar);
-        const uint32_t xdst = ptx::smem_u32(xs + stage * p.x_stage);
-        for (int nb = 0; nb < p.NB; ++nb)
-            ptx::tma_load_2d(xdst + nb * xbs, &tm_x, r0 + nb * 64, b * T, bar);
-        ptx::tma_load_2d(xdst + p.x_dt, &tm_dt, hf8, b * T, bar);
+        const uint32_t fb = bar(B_FULL + s);
+        ptx::mbar_expect_tx(fb, tx_bytes);
+        const uint32_t dst = ptx::smem_u32(h0s + s * h0_stage_bytes);
+        for (int kb = 0; kb < 4; ++kb) ptx::tma_load_2d(dst + kb * RB * 128, &tm_h0, kb * 32, b * HP + r0, fb);
+        const uint32_t xdst = ptx::smem_u32(xs + s * p.x_stage);
+        for (int nb = 0; nb < p.NB; ++nb) ptx::tma_load_2d(xdst + nb * xbs, &tm_x, r0 + nb * 64, b * T, fb);
+        ptx::tma_load_2d(xdst + p.x_dt, &tm_dt, hf8, b * T, fb);
+        loads_issued = k + 1;
     };
 
-    int t = next_valid(start);
-    if (tid == 0 && t < end) issue_load(t, 0);
     int cur_key = -1, cur_b = -1;
     uint32_t k = 0;
-    bool pending_load = (t < end);
-
-    while (t < end) {
-        const int b = t / p.tps, r0 = (t % p.tps) * RB;
+    for (int t = start; t < end; ++t) {
+        const int b = t / p.tps;
+        if (!__ldg(&p.tree.ok[b])) continue;                     // invalid tree: skipped by every role
+        const int r0 = (t % p.tps) * RB;
         const int hfirst = r0 / P;
         const int g = hfirst / hpg;
         const int key = b * G + g;
-        const int stage = k & 1;
+        const int s = k & 1;
         const __nv_bfloat16 *Bseq = p.B + ((size_t)b * T * G + g) * kDstate;   // row j at + j * G * 128
         const size_t brow = (size_t)G * kDstate;
+        bool produced = false;
 
-        // ---------------------------------------------------- per (sequence, group)
+        // ------------------------------------------------------------ (sequence, group) switch
         if (key != cur_key) {
+            if (warp == kProducerWarp && lane == 0) {          // keep the stream going meanwhile
+                produce(k, t);
+                produced = true;
+            }
+            __syncthreads();                                   // every earlier tile is finished
             const bool new_b = (b != cur_b);
             for (int q = tid; q < T_pad * 32; q += kThreads) {
                 const int i = q >> 5, c = q & 31;
@@ -269,7 +336,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             if (new_b) {
                 for (int q = tid; q < T * W; q += kThreads) ancs[q] = __ldg(&p.tree.anc[(size_t)b * T * W + q]);
-                for (uint32_t o = tid * 16u; o < (uint32_t)p.hpt * p.mh_head; o += kThreads * 16u)
+                for (uint32_t o = tid * 16u; o < (uint32_t)hpt * p.mh_head; o += kThreads * 16u)
                     *reinterpret_cast<float4 *>(mh + o) = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (tid == 0) {
                     int len = 0, state = 0;
@@ -326,188 +393,183 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 if (tid == 0) {
                     poff[0] = 0;
                     int total = 0;
-                    for (int w = 0; w < kThreads / 32; ++w) total += misc[M_WSUM + w];
+                    for (int w = 0; w < kWarps; ++w) total += misc[M_WSUM + w];
                     misc[M_TOTAL] = total;
                     misc[M_INSMEM] = total <= p.pair_cap;
                 }
                 cur_b = b;
             }
             __syncthreads();
-            {
-                const int len = min(misc[M_LEN], kPathRows);
-                if (misc[M_STATE])
-                    for (int q = tid; q < len * 16; q += kThreads)
-                        reinterpret_cast<uint4 *>(Bp)[q] =
-                            __ldg(reinterpret_cast<const uint4 *>(Bseq + (size_t)pnode[q >> 4] * brow) + (q & 15));
+            if (misc[M_STATE]) {
+                const int nrows = min((int)misc[M_LEN], kPathRows);
+                for (int q = tid; q < nrows * 32; q += kThreads) {
+                    float b0, b1, b2, b3;
+                    unpack4(__ldg(reinterpret_cast<const uint2 *>(Bseq + (size_t)pnode[q >> 5] * brow) + (q & 31)),
+                            b0, b1, b2, b3);
+                    reinterpret_cast<float4 *>(Bp)[q] = make_float4(b0, b1, b2, b3);
+                }
             }
             if (misc[M_INSMEM]) {
                 const int total = misc[M_TOTAL];
                 for (int q = tid; q < total; q += kThreads) {
-                    int lo = 0, hi = T;                   // poff[lo] <= q < poff[hi]
-                    while (hi - lo > 1) {
-                        const int mid = (lo + hi) >> 1;
-                        if (poff[mid] <= q) lo = mid; else hi = mid;
-                    }
-                    const int j = nth_set_bit(ancs + lo * W, W, q - poff[lo]);
+                    const int i = pair_row(poff, T, q);
+                    const int j = nth_set_bit(ancs + i * W, W, q - poff[i]);
                     pj[q] = (uint8_t)j;
-                    pcb[q] = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, lo);
+                    pcb[q] = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i);
                 }
             }
             ptx::fence_proxy_async_smem();
             __syncthreads();
             cur_key = key;
         }
-
-        const int nt = next_valid(t + 1);
-        uint8_t *h0t = h0s + stage * h0_stage_bytes;
-        uint8_t *xt = xs + stage * p.x_stage;
-
-        // ---------------------------------------------------- root MMA + prefetch (one thread)
-        if (tid == 0) {
-            if (!ptx::mbar_wait(bar_full0 + 8u * stage, (k >> 1) & 1)) {
-                latch_error(p.err, STREE_ERR_TIMEOUT, b, r0, 1);
-                misc[M_ABORT] = 1;
-            } else {
-                pending_load = false;
-                ptx::tc_fence_after();
-                const uint32_t a0 = ptx::smem_u32(h0t);
-                const uint32_t b0 = ptx::smem_u32(cs);
-#pragma unroll
-                for (int kb = 0; kb < 4; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        ptx::mma_tf32(tmem, ptx::desc_kmajor_sw128(a0 + kb * RB * 128 + kk * 32),
-                                      ptx::desc_kmajor_sw128(b0 + kb * T_pad * 128 + kk * 32), idesc_root,
-                                      (kb | kk) != 0);
-                if (nt < end) {
-                    ptx::bulk_wait_read_all();            // tile k-1's stores have left the other stage
-                    issue_load(nt, stage ^ 1);
-                    pending_load = true;
-                }
-            }
-        }
-        __syncthreads();
-        if (misc[M_ABORT]) break;
-
-        // ---------------------------------------------------- per-tile coefficients
-        const int hpt = p.hpt;
         const int len = misc[M_LEN];
         const bool commit = p.do_commit && misc[M_STATE];
-        {
-            const __nv_bfloat16 *dtt = reinterpret_cast<const __nv_bfloat16 *>(xt + p.x_dt);
-            const int hoff = hfirst - (hfirst & ~7);
-            for (int q = tid; q < hpt * T; q += kThreads) {
-                const int hh = q / T, i = q - hh * T;
-                dts[q] = bf2f(dtt[i * p.dt_box + hoff + hh]);
-            }
-        }
-        __syncthreads();
-        for (int q = tid; q < hpt * T; q += kThreads) {
-            const int hh = q / T, i = q - hh * T;
-            float s = 0.f;
-            for (int w = 0; w < W; ++w) {
-                uint32_t bits = ancs[i * W + w];
-                while (bits) {
-                    const int j = (w << 5) + __ffs(bits) - 1;
-                    bits &= bits - 1;
-                    s += dts[hh * T + j];
+        uint8_t *h0t = h0s + s * h0_stage_bytes;
+        uint8_t *xt = xs + s * p.x_stage;
+
+        if (warp == kProducerWarp) {
+            // ------------------------------------------------------------ producer
+            if (lane == 0 && !produced) produce(k, t);
+        } else if (warp == kMmaWarp) {
+            // ------------------------------------------------------------ MMA issue
+            if (lane == 0) {
+                const int a = k & 1;
+                const uint32_t acc = tmem + (uint32_t)(a * p.acc_cols);
+                bool ok = wait(bar(B_FULL + s), (k >> 1) & 1, 20);
+                if (ok && k >= 2) ok = wait(bar(B_ACCE + a), ((k >> 1) - 1) & 1, 21);
+                if (ok) {
+                    ptx::tc_fence_after();
+                    const uint32_t a0 = ptx::smem_u32(h0t), b0 = ptx::smem_u32(cs);
+                    const uint32_t idesc_root = ptx::idesc_tf32(128, T_pad);
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            ptx::mma_tf32(acc, ptx::desc_kmajor_sw128(a0 + kb * RB * 128 + kk * 32),
+                                          ptx::desc_kmajor_sw128(b0 + kb * T_pad * 128 + kk * 32), idesc_root,
+                                          (kb | kk) != 0);
+                    ok = wait(bar(B_MHF), k & 1, 22);
+                }
+                if (ok) {
+                    ptx::tc_fence_after();
+                    const uint32_t xa = ptx::smem_u32(xt);
+                    const uint32_t idesc_tree = ptx::idesc_bf16_amn(128, T_pad);
+                    for (int hh = 0; hh < hpt; ++hh) {
+                        const uint32_t mb = ptx::smem_u32(mh + hh * p.mh_head);
+                        const uint32_t dcol = acc + (uint32_t)(T_pad * (1 + hh));
+                        for (int ks = 0; ks < T_pad / 16; ++ks)
+                            ptx::mma_f16(dcol, ptx::desc_mnmajor_sw128(xa + ks * 2048, xbs, 1024),
+                                         ptx::desc_kmajor_sw128(mb + (ks >> 2) * T_pad * 128 + (ks & 3) * 32),
+                                         idesc_tree, ks != 0);
+                    }
+                    ptx::mma_commit(bar(B_ACCF + a));
+                    ptx::mma_commit(bar(B_MHE));
                 }
             }
-            const float L = __ldg(&p.A[hfirst + hh]) * s;
-            Ls[q] = L;
-            eLs[q] = expf(L);
-        }
-        __syncthreads();
-        // Masked decay matrix of every head of the tile (bf16, K-major swizzled):
-        // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i.
-        {
-            const int total = misc[M_TOTAL];
-            const bool insmem = misc[M_INSMEM] != 0;
-            for (int q = tid; q < hpt * total; q += kThreads) {
-                const int hh = q / total, qq = q - hh * total;
-                int i, j;
-                float cbv;
-                if (insmem) {
-                    int lo = 0, hi = T;
-                    while (hi - lo > 1) {
-                        const int mid = (lo + hi) >> 1;
-                        if (poff[mid] <= qq) lo = mid; else hi = mid;
-                    }
-                    i = lo;
-                    j = pj[qq];
-                    cbv = pcb[qq];
-                } else {
-                    int lo = 0, hi = T;
-                    while (hi - lo > 1) {
-                        const int mid = (lo + hi) >> 1;
-                        if (poff[mid] <= qq) lo = mid; else hi = mid;
-                    }
-                    i = lo;
-                    j = nth_set_bit(ancs + i * W, W, qq - poff[i]);
-                    cbv = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i);
+        } else if (warp < kEpiWarp0) {
+            // ------------------------------------------------------------ prep warps
+            const int ptid = tid - kPrepWarp0 * 32;
+            const int c = k & 1;
+            bool ok = wait(bar(B_FULL + s), (k >> 1) & 1, 30);
+            if (ok && k >= 2) ok = wait(bar(B_COEFE + c), ((k >> 1) - 1) & 1, 31);
+            float *dts = coef(c, 0), *Ls = coef(c, 1), *eLs = coef(c, 2), *wts = coef(c, 3);
+            float *alpha = coef(c, 4);
+            if (ok) {
+                const __nv_bfloat16 *dtt = reinterpret_cast<const __nv_bfloat16 *>(xt + p.x_dt);
+                const int hoff = hfirst - (hfirst & ~7);
+                for (int q = ptid; q < hpt * T; q += kPrepThreads) {
+                    const int hh = q / T, i = q - hh * T;
+                    dts[q] = bf2f(dtt[i * p.dt_box + hoff + hh]);
                 }
-                const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * cbv * dts[hh * T + j];
-                *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) = __float2bfloat16_rn(m);
             }
-        }
-        if (commit) {
-            const int leaf = len > 0 ? pnode[len - 1] : 0;
-            for (int q = tid; q < hpt * len; q += kThreads) {
-                const int hh = q / len, kk = q - hh * len;
-                const int j = pnode[kk];
-                wts[hh * T + kk] = expf(Ls[hh * T + leaf] - Ls[hh * T + j]) * dts[hh * T + j];
+            named_sync(kBarPrep, kPrepThreads);
+            if (ok && !misc[M_ABORT]) {
+                for (int q = ptid; q < hpt * T; q += kPrepThreads) {
+                    const int hh = q / T, i = q - hh * T;
+                    float sum = 0.f;
+                    for (int w = 0; w < W; ++w) {
+                        uint32_t bits = ancs[i * W + w];
+                        while (bits) {
+                            const int j = (w << 5) + __ffs(bits) - 1;
+                            bits &= bits - 1;
+                            sum += dts[hh * T + j];
+                        }
+                    }
+                    const float L = __ldg(&p.A[hfirst + hh]) * sum;
+                    Ls[q] = L;
+                    eLs[q] = expf(L);
+                }
             }
-            if (tid < hpt) alpha[tid] = len > 0 ? eLs[tid * T + leaf] : 1.f;
-        }
-        ptx::fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------------------------------------------- tree MMAs (one thread)
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            const uint32_t xa = ptx::smem_u32(xt);
-            for (int hh = 0; hh < hpt; ++hh) {
-                const uint32_t mb = ptx::smem_u32(mh + hh * p.mh_head);
-                const uint32_t dcol = tmem + (uint32_t)(T_pad * (1 + hh));
-                for (int ks = 0; ks < T_pad / 16; ++ks)
-                    ptx::mma_f16(dcol, ptx::desc_mnmajor_sw128(xa + ks * 2048, xbs, 1024),
-                                 ptx::desc_kmajor_sw128(mb + (ks >> 2) * T_pad * 128 + (ks & 3) * 32), idesc_tree,
-                                 ks != 0);
+            named_sync(kBarPrep, kPrepThreads);
+            if (ok && !misc[M_ABORT]) {
+                if (commit) {
+                    const int leaf = len > 0 ? pnode[len - 1] : 0;
+                    for (int q = ptid; q < hpt * len; q += kPrepThreads) {
+                        const int hh = q / len, kk = q - hh * len;
+                        const int j = pnode[kk];
+                        wts[hh * T + kk] = expf(Ls[hh * T + leaf] - Ls[hh * T + j]) * dts[hh * T + j];
+                    }
+                    if (ptid < hpt) alpha[ptid] = len > 0 ? eLs[ptid * T + leaf] : 1.f;
+                }
+                mbar_arrive(bar(B_COEFF + c));
+                // Masked decay matrix of every head of the tile (bf16, K-major swizzled):
+                // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i.
+                ok = (k == 0) || wait(bar(B_MHE), (k - 1) & 1, 32);
+                if (ok) {
+                    const int total = misc[M_TOTAL];
+                    const bool insmem = misc[M_INSMEM] != 0;
+                    for (int q = ptid; q < hpt * total; q += kPrepThreads) {
+                        const int hh = q / total, qq = q - hh * total;
+                        const int i = pair_row(poff, T, qq);
+                        int j;
+                        float cbv;
+                        if (insmem) {
+                            j = pj[qq];
+                            cbv = pcb[qq];
+                        } else {
+                            j = nth_set_bit(ancs + i * W, W, qq - poff[i]);
+                            cbv = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i);
+                        }
+                        const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * cbv * dts[hh * T + j];
+                        *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
+                            __float2bfloat16_rn(m);
+                    }
+                    ptx::fence_proxy_async_smem();
+                    mbar_arrive(bar(B_MHF));
+                }
             }
-            ptx::mma_commit(bar_mma);
-        }
-
-        // ---------------------------------------------------- wait for the MMAs
-        if (!ptx::mbar_wait(bar_mma, k & 1)) {
-            latch_error(p.err, STREE_ERR_TIMEOUT, b, r0, 2);
-            misc[M_ABORT] = 1;
-        }
-        __syncthreads();
-        if (misc[M_ABORT]) break;
-        ptx::tc_fence_after();
-
-        // ---------------------------------------------------- commit, in place over h0
-        if (commit) {
-            const int tpr = kThreads / RB;                 // threads per row
-            const int row = tid % RB, part = tid / RB;
-            const int hh = (r0 + row) / P - hfirst;
-            if (tpr == 2)
-                commit_rows<64>(h0t, xt, xbs, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 64);
-            else
-                commit_rows<32>(h0t, xt, xbs, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 32);
-        }
-        __syncthreads();                                   // x rows of the path are read
-
-        // ---------------------------------------------------- y, in place over x
-        {
-            const int quad = warp & 3, half = warp >> 2;
-            if (quad * 32 < RB) {
+        } else {
+            // ------------------------------------------------------------ epilogue warps
+            const int etid = tid - kEpiWarp0 * 32, ewarp = warp - kEpiWarp0;
+            const int a = k & 1, c = k & 1;
+            bool ok = wait(bar(B_FULL + s), (k >> 1) & 1, 40);
+            if (ok) ok = wait(bar(B_COEFF + c), (k >> 1) & 1, 41);
+            if (ok) ok = wait(bar(B_ACCF + a), (k >> 1) & 1, 42);
+            named_sync(kBarEpi, kEpiThreads);
+            // Warp-uniform decision: tcgen05.ld below is a warp-collective instruction.
+            const bool run = __all_sync(0xffffffffu, ok && !misc[M_ABORT]);
+            if (run) ptx::tc_fence_after();
+            const float *eLs = coef(c, 2), *wts = coef(c, 3), *alpha = coef(c, 4);
+            if (run && commit) {
+                const int tpr = kEpiThreads / RB;                  // threads per row: 2 or 4
+                const int row = etid % RB, part = etid / RB;
+                const int hh = (r0 + row) / P - hfirst;
+                const MnCol xc(row, xbs);
+                if (tpr == 2)
+                    commit_rows<64>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 64);
+                else
+                    commit_rows<32>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 32);
+            }
+            named_sync(kBarEpi, kEpiThreads);                  // x rows of the path are read
+            const int quad = ewarp & 3, half = ewarp >> 2;
+            if (run && quad * 32 < RB) {
                 const int row = quad * 32 + lane;
-                const int hh = (r0 + row) / P - hfirst;   // same for the whole warp (P >= 32)
+                const int hh = (r0 + row) / P - hfirst;           // same for the whole warp (P >= 32)
                 const float Dh = __ldg(&p.D[hfirst + hh]);
                 const float *eLh = eLs + hh * T;
-                const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+                const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * p.acc_cols);
                 const uint32_t ty = tl + (uint32_t)(T_pad * (1 + hh));
+                const MnCol xc(row, xbs);
                 for (int c0 = half * 16; c0 < T; c0 += 32) {
                     float R[16], Y[16];
                     ptx::tmem_ld16(tl + (uint32_t)c0, R);
@@ -516,45 +578,46 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     for (int u = 0; u < 16; ++u) {
                         const int i = c0 + u;
                         if (i < T) {
-                            __nv_bfloat16 *xe = reinterpret_cast<__nv_bfloat16 *>(xt + mn_off(i, row, xbs));
-                            const float yv = fmaf(eLh[i], R[u], fmaf(Dh, bf2f(*xe), Y[u]));
-                            *xe = __float2bfloat16_rn(yv);
+                            __nv_bfloat16 *xe = reinterpret_cast<__nv_bfloat16 *>(xt + xc.at(i));
+                            *xe = __float2bfloat16_rn(fmaf(eLh[i], R[u], fmaf(Dh, bf2f(*xe), Y[u])));
                         }
                     }
                 }
             }
-        }
-        ptx::tc_fence_before();
-        ptx::fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---------------------------------------------------- stores (one thread)
-        if (tid == 0) {
-            const uint32_t xsrc = ptx::smem_u32(xt);
-            for (int nb = 0; nb < p.NB; ++nb)
-                ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
-            if (commit) {
-                const uint32_t src = ptx::smem_u32(h0t);
-                for (int kb = 0; kb < 4; ++kb)
-                    ptx::tma_store_2d(&tm_hn, kb * 32, b * HP + r0, src + kb * RB * 128);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (run && lane == 0) {
+                mbar_arrive(bar(B_ACCE + a));
+                mbar_arrive(bar(B_COEFE + c));
             }
-            ptx::bulk_commit();
+            ptx::fence_proxy_async_smem();
+            named_sync(kBarEpi, kEpiThreads);
+            if (run && etid == 0) {
+                const uint32_t xsrc = ptx::smem_u32(xt);
+                for (int nb = 0; nb < p.NB; ++nb) ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
+                if (commit) {
+                    const uint32_t src = ptx::smem_u32(h0t);
+                    for (int kb = 0; kb < 4; ++kb) ptx::tma_store_2d(&tm_hn, kb * 32, b * HP + r0, src + kb * RB * 128);
+                }
+                ptx::bulk_commit();
+                ptx::bulk_wait_read_all();
+                mbar_arrive(bar(B_EMPTY + s));
+            }
         }
         ++k;
-        t = nt;
     }
 
-    if (tid == 0) {
-        ptx::bulk_wait_all();
-        if (misc[M_ABORT] && pending_load) {
-            // A load may still land in this CTA's shared memory: give it a bounded wait.
-            ptx::mbar_wait(bar_full0 + 8u * (k & 1), (k >> 1) & 1);
-            ptx::mbar_wait(bar_full0 + 8u * ((k + 1) & 1), ((k + 1) >> 1) & 1);
-        }
+    // ---------------------------------------------------------------- teardown
+    if (warp == kEpiWarp0 && lane == 0) ptx::bulk_wait_all();
+    if (warp == kProducerWarp && lane == 0 && misc[M_ABORT]) {
+        // Loads issued but never consumed may still land in this CTA's shared
+        // memory: give the last two a bounded wait before the CTA exits.
+        for (uint32_t q = loads_issued >= 2 ? loads_issued - 2 : 0; q < loads_issued; ++q)
+            ptx::mbar_wait(bar(B_FULL + (q & 1)), (q >> 1) & 1);
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, p.tmem_cols);
     }
@@ -618,16 +681,13 @@ bool layout(const ScanArgs &a, int RB, TcParams &p, size_t &smem)
     p.off_mh = round_up(off, 1024u);
     p.mh_head = (uint32_t)KA * T_pad * 128u;
     off = p.off_mh + (uint32_t)hpt * p.mh_head;
-    p.off_bp = round_up(off, 16u);     off = p.off_bp + (uint32_t)kPathRows * kDstate * 2u;
+    p.off_bp = round_up(off, 16u);     off = p.off_bp + (uint32_t)kPathRows * kDstate * 4u;
     p.off_anc = round_up(off, 16u);    off = p.off_anc + (uint32_t)T * W * 4u;
     p.off_poff = round_up(off, 16u);   off = p.off_poff + (uint32_t)(T + 1) * 4u;
-    p.off_dts = round_up(off, 16u);    off = p.off_dts + (uint32_t)hpt * T * 4u;
-    p.off_L = round_up(off, 16u);      off = p.off_L + (uint32_t)hpt * T * 4u;
-    p.off_eL = round_up(off, 16u);     off = p.off_eL + (uint32_t)hpt * T * 4u;
-    p.off_w = round_up(off, 16u);      off = p.off_w + (uint32_t)hpt * T * 4u;
-    p.off_alpha = round_up(off, 16u);  off = p.off_alpha + (uint32_t)hpt * 4u;
+    p.coef_slot = round_up((uint32_t)(4 * hpt * T + hpt) * 4u, 16u);
+    p.off_coef = round_up(off, 16u);   off = p.off_coef + 2u * p.coef_slot;
     p.off_pnode = round_up(off, 16u);  off = p.off_pnode + (uint32_t)T * 2u;
-    p.off_bar = round_up(off, 16u);    off = p.off_bar + 3u * 8u;
+    p.off_bar = round_up(off, 16u);    off = p.off_bar + kNumBars * 8u;
     p.off_misc = round_up(off, 16u);   off = p.off_misc + kMiscWords * 4u;
     p.off_pcb = round_up(off, 16u);
     const size_t fixed = (size_t)p.off_pcb + 1024;            // + alignment slack of the dynamic base
@@ -646,8 +706,9 @@ bool layout(const ScanArgs &a, int RB, TcParams &p, size_t &smem)
     p.RB = RB;
     p.NB = NB;
     p.hpt = hpt;
+    p.acc_cols = (1 + hpt) * T_pad;
     uint32_t cols = 32;
-    while (cols < (uint32_t)((1 + hpt) * T_pad)) cols <<= 1;
+    while (cols < (uint32_t)(2 * p.acc_cols)) cols <<= 1;
     if (cols > 512) return false;
     p.tmem_cols = cols;
     return true;
