@@ -46,15 +46,21 @@ constexpr int kDtBox = 16;                 // heads per dt box (32 bytes of bf16
 constexpr int kPathRows = 8;               // accepted-path rows of B staged in smem (fp32)
 constexpr size_t kSmemLimit = 232448;      // 227 KB opt-in dynamic shared memory
 
-constexpr int kProducerWarp = 0, kMmaWarp = 1, kPrepWarp0 = 2, kPrepWarps = 2, kEpiWarp0 = 4, kEpiWarps = 8;
+constexpr int kProducerWarp = 0, kMmaWarp = 1, kPrepWarp0 = 2, kPrepWarps = 4, kEpiWarp0 = 6, kEpiWarps = 8;
+constexpr int kMaxStages = 3;
+constexpr int kMaxSmemHeads = 1024;        // A and D are staged in shared memory
 constexpr int kWarps = kEpiWarp0 + kEpiWarps;
 constexpr int kThreads = kWarps * 32;
 constexpr int kPrepThreads = kPrepWarps * 32, kEpiThreads = kEpiWarps * 32;
 constexpr int kBarEpi = 1, kBarPrep = 2;   // named barriers (0 is __syncthreads)
 
-enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_WSUM = 8, kMiscWords = 8 + kWarps };
-enum Bars { B_FULL = 0, B_EMPTY = 2, B_ACCF = 4, B_ACCE = 6, B_MHF = 8, B_MHE = 9, B_COEFF = 10, B_COEFE = 12,
-            kNumBars = 14 };
+enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_SDESC = 8, M_WSUM = 8 + 2 * kMaxStages,
+            kMiscWords = M_WSUM + kWarps };
+// mbarriers: TMA stage full / epilogue done with a stage (ring of S), tensor-memory
+// accumulator full / empty (ring of 2), masked-decay matrix full / empty, and
+// per-tile coefficients full / empty (ring of 2).
+enum Bars { B_FULL = 0, B_EPID = kMaxStages, B_ACCF = 2 * kMaxStages, B_ACCE = B_ACCF + 2, B_MHF = B_ACCE + 2,
+            B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, kNumBars = B_COEFE + 2 };
 
 struct TcParams {
     const __nv_bfloat16 *__restrict__ B;
@@ -65,10 +71,10 @@ struct TcParams {
     const int32_t *__restrict__ path_len;
     TreeView tree;
     int32_t *err;
-    int T, T_pad, KA, H, P, G, RB, NB, tps, ntiles, maxlen, do_commit, hpt, pair_cap, dt_box, acc_cols;
+    int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, hpt, pair_cap, dt_box, acc_cols;
     uint32_t tmem_cols;
     uint32_t off_x, x_dt, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_coef, coef_slot,
-        off_pnode, off_bar, off_misc, off_pcb, off_pj;
+        off_pnode, off_bar, off_misc, off_ad, off_pcb, off_pj, off_pi;
 };
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -115,6 +121,29 @@ __device__ __forceinline__ float dot_cb(const uint8_t *cs, int T_pad, const __nv
         const float4 cv = *reinterpret_cast<const float4 *>(crow + (c >> 3) * T_pad * 128 + (((c & 7) ^ (i & 7)) << 4));
         float b0, b1, b2, b3;
         unpack4(__ldg(brow + c), b0, b1, b2, b3);
+        acc = fmaf(cv.x, b0, acc);
+        acc = fmaf(cv.y, b1, acc);
+        acc = fmaf(cv.z, b2, acc);
+        acc = fmaf(cv.w, b3, acc);
+    }
+    return acc;
+}
+
+// C_i . B_j over the quarter `part` (32 of the 128 state columns); four lanes of
+// a warp combine their parts with shuffles.
+__device__ __forceinline__ float dot_cb_part(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i, int part)
+{
+    float acc = 0.f;
+    const uint8_t *crow = cs + part * T_pad * 128 + i * 128;     // K-atom `part` holds columns 32*part..
+    const uint2 *brow = reinterpret_cast<const uint2 *>(Bj) + part * 8;
+    uint2 raw[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) raw[c] = __ldg(brow + c);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const float4 cv = *reinterpret_cast<const float4 *>(crow + ((c ^ (i & 7)) << 4));
+        float b0, b1, b2, b3;
+        unpack4(raw[c], b0, b1, b2, b3);
         acc = fmaf(cv.x, b0, acc);
         acc = fmaf(cv.y, b1, acc);
         acc = fmaf(cv.z, b2, acc);
@@ -180,17 +209,23 @@ __device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, con
             }
         }
     }
+    float4 h[CPT / 4];
 #pragma unroll
     for (int c = 0; c < CPT / 4; ++c) {
         const int n = c_lo + 4 * c;
         const int kb = n >> 5, ch = (n & 31) >> 2;
-        float4 *ptr = reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
-        float4 v = *ptr;
-        v.x = fmaf(al, v.x, acc[4 * c + 0]);
-        v.y = fmaf(al, v.y, acc[4 * c + 1]);
-        v.z = fmaf(al, v.z, acc[4 * c + 2]);
-        v.w = fmaf(al, v.w, acc[4 * c + 3]);
-        *ptr = v;
+        h[c] = *reinterpret_cast<const float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
+    }
+#pragma unroll
+    for (int c = 0; c < CPT / 4; ++c) {
+        const int n = c_lo + 4 * c;
+        const int kb = n >> 5, ch = (n & 31) >> 2;
+        float4 v;
+        v.x = fmaf(al, h[c].x, acc[4 * c + 0]);
+        v.y = fmaf(al, h[c].y, acc[4 * c + 1]);
+        v.z = fmaf(al, h[c].z, acc[4 * c + 2]);
+        v.w = fmaf(al, h[c].w, acc[4 * c + 3]);
+        *reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
     }
 }
 
@@ -213,11 +248,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = p.T, T_pad = p.T_pad, RB = p.RB, P = p.P, H = p.H, G = p.G, W = p.tree.W, HP = H * P;
-    const int hpg = H / G, hpt = p.hpt;
+    const int hpg = H / G, hpt = p.hpt, S = p.S;
     const uint32_t xbs = (uint32_t)T_pad * 128u;                      // x: bytes per 64-column block
 
-    uint8_t *h0s = smem;                                              // 2 x [4 atoms][RB rows][128 B] fp32
-    uint8_t *xs = smem + p.off_x;                                     // 2 x {NB x [T_pad rows][128 B] x, dt}
+    uint8_t *h0s = smem;                                              // S x [4 atoms][RB rows][128 B] fp32
+    uint8_t *xs = smem + p.off_x;                                     // S x {NB x [T_pad rows][128 B] x, dt}
     uint8_t *cs = smem + p.off_c;                                     // [4 atoms][T_pad rows][128 B] fp32
     uint8_t *mh = smem + p.off_mh;                                    // hpt x [KA atoms][T_pad rows][128 B] bf16
     float *Bp = reinterpret_cast<float *>(smem + p.off_bp);           // [kPathRows][128] fp32
@@ -226,8 +261,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     int16_t *pnode = reinterpret_cast<int16_t *>(smem + p.off_pnode); // [T]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     volatile int32_t *misc = reinterpret_cast<volatile int32_t *>(smem + p.off_misc);
-    float *pcb = reinterpret_cast<float *>(smem + p.off_pcb);         // [pair_cap]
-    uint8_t *pj = smem + p.off_pj;                                    // [pair_cap]
+    float *Ash = reinterpret_cast<float *>(smem + p.off_ad);          // [H] A, then [H] D
+    float *Dsh = Ash + H;
+    float *pcb = reinterpret_cast<float *>(smem + p.off_pcb);         // [pair_cap] C_i . B_j
+    uint8_t *pj = smem + p.off_pj;                                    // [pair_cap] j
+    uint8_t *pi = smem + p.off_pi;                                    // [pair_cap] i
     // Per-tile coefficients, two slots: dts, L, exp(L), commit weights [hpt][T] each, alpha [hpt].
     auto coef = [&](int slot, int which) {
         return reinterpret_cast<float *>(smem + p.off_coef + slot * p.coef_slot) + which * hpt * T;
@@ -243,9 +281,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         ptx::prefetch_tensormap(&tm_dt);
         ptx::prefetch_tensormap(&tm_hn);
         ptx::prefetch_tensormap(&tm_y);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             ptx::mbar_init(bar(B_FULL + s), 1);
-            ptx::mbar_init(bar(B_EMPTY + s), 1);
+            ptx::mbar_init(bar(B_EPID + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(bar(B_ACCF + s), 1);
             ptx::mbar_init(bar(B_ACCE + s), kEpiWarps);
             ptx::mbar_init(bar(B_COEFF + s), kPrepThreads);
@@ -256,10 +296,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         ptx::fence_mbar_init();
         for (int q = 0; q < kMiscWords; ++q) misc[q] = 0;
     }
+    __syncthreads();                                  // misc cleared before the allocation writes it
     // Operand rows the MMAs read past the valid tile (rows >= RB, nodes >= T)
     // must hold finite values: clear the staging regions once.
     for (uint32_t o = tid * 16u; o < p.off_mh; o += kThreads * 16u)
         *reinterpret_cast<float4 *>(smem + o) = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int h = tid; h < H; h += kThreads) {
+        Ash[h] = __ldg(&p.A[h]);
+        Dsh[h] = __ldg(&p.D[h]);
+    }
     if (warp == kMmaWarp) {
         ptx::tmem_alloc(ptx::smem_u32(const_cast<int32_t *>(&misc[M_TMEM])), p.tmem_cols);
         ptx::tmem_relinquish();
@@ -282,11 +327,30 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
 
     const int start = (int)((long long)blockIdx.x * p.ntiles / gridDim.x);
     const int end = (int)((long long)(blockIdx.x + 1) * p.ntiles / gridDim.x);
-    uint32_t loads_issued = 0;
+    uint32_t loads_issued = 0, stores_issued = 0;
 
-    auto produce = [&](uint32_t k, int t) {                    // producer warp, lane 0
-        const int s = k & 1;
-        if (k >= 2 && !wait(bar(B_EMPTY + s), ((k >> 1) - 1) & 1, 10)) return;
+    // Producer: TMA stores of tile q once its epilogue is done (descriptor in misc).
+    auto store_tile = [&](uint32_t q) {
+        const int s = q % S;
+        if (!wait(bar(B_EPID + s), (q / S) & 1, 11)) return;
+        const int t = misc[M_SDESC + 2 * s], commit = misc[M_SDESC + 2 * s + 1];
+        const int b = t / p.tps, r0 = (t % p.tps) * RB;
+        const uint32_t xsrc = ptx::smem_u32(xs + s * p.x_stage);
+        for (int nb = 0; nb < p.NB; ++nb) ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
+        if (commit) {
+            const uint32_t src = ptx::smem_u32(h0s + s * h0_stage_bytes);
+            for (int kb = 0; kb < 4; ++kb) ptx::tma_store_2d(&tm_hn, kb * 32, b * HP + r0, src + kb * RB * 128);
+        }
+        ptx::bulk_commit();
+        stores_issued = q + 1;
+    };
+    // Producer: TMA loads of tile k into stage k % S once tile k - S has left it.
+    auto produce = [&](uint32_t k, int t) {
+        const int s = k % S;
+        if (k >= (uint32_t)S) {
+            store_tile(k - S);
+            ptx::bulk_wait_read_all();
+        }
         if (misc[M_ABORT]) return;
         const int b = t / p.tps, r0 = (t % p.tps) * RB;
         const int hf8 = (r0 / P) & ~7;
@@ -309,7 +373,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         const int hfirst = r0 / P;
         const int g = hfirst / hpg;
         const int key = b * G + g;
-        const int s = k & 1;
+        const int s = k % S;
+        const uint32_t sph = (k / S) & 1;                        // phase parity of this stage use
         const __nv_bfloat16 *Bseq = p.B + ((size_t)b * T * G + g) * kDstate;   // row j at + j * G * 128
         const size_t brow = (size_t)G * kDstate;
         bool produced = false;
@@ -320,8 +385,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 produce(k, t);
                 produced = true;
             }
-            __syncthreads();                                   // every earlier tile is finished
+            __syncthreads();                                   // every earlier tile is consumed
             const bool new_b = (b != cur_b);
+            // Phase 1: independent loads.
             for (int q = tid; q < T_pad * 32; q += kThreads) {
                 const int i = q >> 5, c = q & 31;
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -339,43 +405,38 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 for (uint32_t o = tid * 16u; o < (uint32_t)hpt * p.mh_head; o += kThreads * 16u)
                     *reinterpret_cast<float4 *>(mh + o) = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (tid == 0) {
-                    int len = 0, state = 0;
-                    if (p.do_commit) {
-                        len = __ldg(&p.path_len[b]);
-                        state = 1;
-                        if (len < 0 || len > p.maxlen || len > T) {
-                            state = 0;
-                            latch_error(p.err, STREE_ERR_BAD_PATH, b, -1, len);
-                        } else if (len > 0) {
-                            const int leaf = __ldg(&p.path[(size_t)b * p.maxlen + len - 1]);
-                            if (leaf < 0 || leaf >= T || __ldg(&p.tree.depth[(size_t)b * T + leaf]) != len - 1) {
-                                state = 0;
-                                latch_error(p.err, STREE_ERR_BAD_PATH, b, len - 1, leaf);
-                            }
-                        }
-                    }
-                    misc[M_LEN] = len;
-                    misc[M_STATE] = state;
+                    misc[M_LEN] = p.do_commit ? __ldg(&p.path_len[b]) : 0;
+                    misc[M_STATE] = p.do_commit;
                 }
             }
             __syncthreads();
             if (new_b) {
-                // Every path position q must hold the depth-q ancestor of the last node.
+                // Phase 2: the accepted path -- position q must hold the depth-q ancestor
+                // of the last node -- and the pair offsets (prefix sum of ancestor counts).
                 const int len = misc[M_LEN];
-                if (misc[M_STATE] && len > 0) {
-                    const int leaf = __ldg(&p.path[(size_t)b * p.maxlen + len - 1]);
-                    for (int q = tid; q < len; q += kThreads) {
-                        const int j = __ldg(&p.path[(size_t)b * p.maxlen + q]);
-                        const bool good = j >= 0 && j < T && ((ancs[leaf * W + (j >> 5)] >> (j & 31)) & 1u) &&
-                                          __ldg(&p.tree.depth[(size_t)b * T + j]) == q;
-                        if (!good) {
+                if (p.do_commit) {
+                    if (len < 0 || len > p.maxlen || len > T) {
+                        if (tid == 0) {
                             misc[M_STATE] = 0;
-                            latch_error(p.err, STREE_ERR_BAD_PATH, b, q, j);
+                            latch_error(p.err, STREE_ERR_BAD_PATH, b, -1, len);
                         }
-                        pnode[q] = (int16_t)(good ? j : 0);
+                    } else if (len > 0) {
+                        const int leaf = __ldg(&p.path[(size_t)b * p.maxlen + len - 1]);
+                        const bool leaf_ok = leaf >= 0 && leaf < T;
+                        for (int q = tid; q < len; q += kThreads) {
+                            const int j = __ldg(&p.path[(size_t)b * p.maxlen + q]);
+                            const bool good = leaf_ok && j >= 0 && j < T &&
+                                              ((ancs[leaf * W + (j >> 5)] >> (j & 31)) & 1u) &&
+                                              __ldg(&p.tree.depth[(size_t)b * T + j]) == q &&
+                                              (q != len - 1 || __ldg(&p.tree.depth[(size_t)b * T + leaf]) == len - 1);
+                            if (!good) {
+                                misc[M_STATE] = 0;
+                                latch_error(p.err, STREE_ERR_BAD_PATH, b, q, j);
+                            }
+                            pnode[q] = (int16_t)(good ? j : 0);
+                        }
                     }
                 }
-                // Pair offsets: exclusive prefix sum of the ancestor counts (T <= 128).
                 int cnt = 0;
                 if (tid < T)
                     for (int w = 0; w < W; ++w) cnt += __popc(ancs[tid * W + w]);
@@ -400,6 +461,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 cur_b = b;
             }
             __syncthreads();
+            // Phase 3: path rows of B (fp32) for the commit, C_i . B_j of every ancestor pair.
             if (misc[M_STATE]) {
                 const int nrows = min((int)misc[M_LEN], kPathRows);
                 for (int q = tid; q < nrows * 32; q += kThreads) {
@@ -411,11 +473,29 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             if (misc[M_INSMEM]) {
                 const int total = misc[M_TOTAL];
-                for (int q = tid; q < total; q += kThreads) {
-                    const int i = pair_row(poff, T, q);
-                    const int j = nth_set_bit(ancs + i * W, W, q - poff[i]);
-                    pj[q] = (uint8_t)j;
-                    pcb[q] = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i);
+                // Node i's pairs: its ancestors in increasing order.
+                for (int i = tid; i < T; i += kThreads) {
+                    int q = poff[i];
+                    for (int w = 0; w < W; ++w) {
+                        uint32_t bits = ancs[i * W + w];
+                        while (bits) {
+                            pj[q] = (uint8_t)((w << 5) + __ffs(bits) - 1);
+                            pi[q] = (uint8_t)i;
+                            bits &= bits - 1;
+                            ++q;
+                        }
+                    }
+                }
+                __syncthreads();
+                // Four lanes per pair, a quarter of the state columns each.
+                const int part = lane & 3;
+                for (int q0 = (tid >> 2); q0 < ((total + 7) & ~7); q0 += kThreads / 4) {
+                    const int q = q0 < total ? q0 : total - 1;
+                    const int i = pi[q], j = pj[q];
+                    float v = dot_cb_part(cs, T_pad, Bseq + (size_t)j * brow, i, part);
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    if (part == 0 && q0 < total) pcb[q] = v;
                 }
             }
             ptx::fence_proxy_async_smem();
@@ -435,7 +515,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             if (lane == 0) {
                 const int a = k & 1;
                 const uint32_t acc = tmem + (uint32_t)(a * p.acc_cols);
-                bool ok = wait(bar(B_FULL + s), (k >> 1) & 1, 20);
+                bool ok = wait(bar(B_FULL + s), sph, 20);
                 if (ok && k >= 2) ok = wait(bar(B_ACCE + a), ((k >> 1) - 1) & 1, 21);
                 if (ok) {
                     ptx::tc_fence_after();
@@ -470,7 +550,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             // ------------------------------------------------------------ prep warps
             const int ptid = tid - kPrepWarp0 * 32;
             const int c = k & 1;
-            bool ok = wait(bar(B_FULL + s), (k >> 1) & 1, 30);
+            bool ok = wait(bar(B_FULL + s), sph, 30);
             if (ok && k >= 2) ok = wait(bar(B_COEFE + c), ((k >> 1) - 1) & 1, 31);
             float *dts = coef(c, 0), *Ls = coef(c, 1), *eLs = coef(c, 2), *wts = coef(c, 3);
             float *alpha = coef(c, 4);
@@ -486,16 +566,16 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             if (ok && !misc[M_ABORT]) {
                 for (int q = ptid; q < hpt * T; q += kPrepThreads) {
                     const int hh = q / T, i = q - hh * T;
+                    const float *dh = dts + hh * T;
                     float sum = 0.f;
                     for (int w = 0; w < W; ++w) {
                         uint32_t bits = ancs[i * W + w];
                         while (bits) {
-                            const int j = (w << 5) + __ffs(bits) - 1;
+                            sum += dh[(w << 5) + __ffs(bits) - 1];
                             bits &= bits - 1;
-                            sum += dts[hh * T + j];
                         }
                     }
-                    const float L = __ldg(&p.A[hfirst + hh]) * sum;
+                    const float L = Ash[hfirst + hh] * sum;
                     Ls[q] = L;
                     eLs[q] = expf(L);
                 }
@@ -517,22 +597,24 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 ok = (k == 0) || wait(bar(B_MHE), (k - 1) & 1, 32);
                 if (ok) {
                     const int total = misc[M_TOTAL];
-                    const bool insmem = misc[M_INSMEM] != 0;
-                    for (int q = ptid; q < hpt * total; q += kPrepThreads) {
-                        const int hh = q / total, qq = q - hh * total;
-                        const int i = pair_row(poff, T, qq);
-                        int j;
-                        float cbv;
-                        if (insmem) {
-                            j = pj[qq];
-                            cbv = pcb[qq];
-                        } else {
-                            j = nth_set_bit(ancs + i * W, W, qq - poff[i]);
-                            cbv = dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i);
+                    if (misc[M_INSMEM]) {
+                        for (int q = ptid; q < hpt * total; q += kPrepThreads) {
+                            const int hh = q / total, qq = q - hh * total;
+                            const int i = pi[qq], j = pj[qq];
+                            const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * pcb[qq] * dts[hh * T + j];
+                            *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
+                                __float2bfloat16_rn(m);
                         }
-                        const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * cbv * dts[hh * T + j];
-                        *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
-                            __float2bfloat16_rn(m);
+                    } else {
+                        for (int q = ptid; q < hpt * total; q += kPrepThreads) {
+                            const int hh = q / total, qq = q - hh * total;
+                            const int i = pair_row(poff, T, qq);
+                            const int j = nth_set_bit(ancs + i * W, W, qq - poff[i]);
+                            const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) *
+                                            dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i) * dts[hh * T + j];
+                            *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
+                                __float2bfloat16_rn(m);
+                        }
                     }
                     ptx::fence_proxy_async_smem();
                     mbar_arrive(bar(B_MHF));
@@ -542,7 +624,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             // ------------------------------------------------------------ epilogue warps
             const int etid = tid - kEpiWarp0 * 32, ewarp = warp - kEpiWarp0;
             const int a = k & 1, c = k & 1;
-            bool ok = wait(bar(B_FULL + s), (k >> 1) & 1, 40);
+            bool ok = wait(bar(B_FULL + s), sph, 40);
             if (ok) ok = wait(bar(B_COEFF + c), (k >> 1) & 1, 41);
             if (ok) ok = wait(bar(B_ACCF + a), (k >> 1) & 1, 42);
             named_sync(kBarEpi, kEpiThreads);
@@ -555,33 +637,33 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 const int row = etid % RB, part = etid / RB;
                 const int hh = (r0 + row) / P - hfirst;
                 const MnCol xc(row, xbs);
-                if (tpr == 2)
-                    commit_rows<64>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 64);
-                else
-                    commit_rows<32>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, part * 32);
+                const int cols = kDstate / tpr;
+                for (int c_lo = part * cols; c_lo < (part + 1) * cols; c_lo += 32)
+                    commit_rows<32>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, c_lo);
             }
             named_sync(kBarEpi, kEpiThreads);                  // x rows of the path are read
-            const int quad = ewarp & 3, half = ewarp >> 2;
+            // A warp reads only its own quarter of the tensor-memory lanes: 32 * (warp % 4).
+            const int quad = warp & 3, half = ewarp >> 2;
             if (run && quad * 32 < RB) {
                 const int row = quad * 32 + lane;
                 const int hh = (r0 + row) / P - hfirst;           // same for the whole warp (P >= 32)
-                const float Dh = __ldg(&p.D[hfirst + hh]);
+                const float Dh = Dsh[hfirst + hh];
                 const float *eLh = eLs + hh * T;
                 const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * p.acc_cols);
                 const uint32_t ty = tl + (uint32_t)(T_pad * (1 + hh));
                 const MnCol xc(row, xbs);
                 for (int c0 = half * 16; c0 < T; c0 += 32) {
-                    float R[16], Y[16];
+                    float R[16], Y[16], X[16];
                     ptx::tmem_ld16(tl + (uint32_t)c0, R);
                     ptx::tmem_ld16(ty + (uint32_t)c0, Y);
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int i = c0 + u;
-                        if (i < T) {
-                            __nv_bfloat16 *xe = reinterpret_cast<__nv_bfloat16 *>(xt + xc.at(i));
-                            *xe = __float2bfloat16_rn(fmaf(eLh[i], R[u], fmaf(Dh, bf2f(*xe), Y[u])));
-                        }
-                    }
+                    for (int u = 0; u < 16; ++u)
+                        X[u] = (c0 + u < T) ? bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(c0 + u))) : 0.f;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        if (c0 + u < T)
+                            *reinterpret_cast<__nv_bfloat16 *>(xt + xc.at(c0 + u)) =
+                                __float2bfloat16_rn(fmaf(eLh[c0 + u], R[u], fmaf(Dh, X[u], Y[u])));
                 }
             }
             ptx::tc_fence_before();
@@ -593,27 +675,24 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             ptx::fence_proxy_async_smem();
             named_sync(kBarEpi, kEpiThreads);
             if (run && etid == 0) {
-                const uint32_t xsrc = ptx::smem_u32(xt);
-                for (int nb = 0; nb < p.NB; ++nb) ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
-                if (commit) {
-                    const uint32_t src = ptx::smem_u32(h0t);
-                    for (int kb = 0; kb < 4; ++kb) ptx::tma_store_2d(&tm_hn, kb * 32, b * HP + r0, src + kb * RB * 128);
-                }
-                ptx::bulk_commit();
-                ptx::bulk_wait_read_all();
-                mbar_arrive(bar(B_EMPTY + s));
+                misc[M_SDESC + 2 * s] = t;                     // the producer issues the stores
+                misc[M_SDESC + 2 * s + 1] = commit ? 1 : 0;
+                mbar_arrive(bar(B_EPID + s));
             }
         }
         ++k;
     }
 
     // ---------------------------------------------------------------- teardown
-    if (warp == kEpiWarp0 && lane == 0) ptx::bulk_wait_all();
-    if (warp == kProducerWarp && lane == 0 && misc[M_ABORT]) {
-        // Loads issued but never consumed may still land in this CTA's shared
-        // memory: give the last two a bounded wait before the CTA exits.
-        for (uint32_t q = loads_issued >= 2 ? loads_issued - 2 : 0; q < loads_issued; ++q)
-            ptx::mbar_wait(bar(B_FULL + (q & 1)), (q >> 1) & 1);
+    if (warp == kProducerWarp && lane == 0) {
+        for (uint32_t q = stores_issued; q < k && !misc[M_ABORT]; ++q) store_tile(q);
+        ptx::bulk_wait_all();
+        if (misc[M_ABORT]) {
+            // Loads issued but never consumed may still land in this CTA's shared
+            // memory: give them a bounded wait before the CTA exits.
+            for (uint32_t q = loads_issued >= (uint32_t)S ? loads_issued - S : 0; q < loads_issued; ++q)
+                ptx::mbar_wait(bar(B_FULL + q % S), (q / S) & 1);
+        }
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -659,18 +738,18 @@ struct TcPlan {
     int grid;
 };
 
-// Shared-memory layout for a tile height RB; returns false if it does not fit.
-bool layout(const ScanArgs &a, int RB, TcParams &p, size_t &smem)
+// Shared-memory layout for a tile height RB and S stages; false if it does not fit.
+bool layout(const ScanArgs &a, int RB, int S, TcParams &p, size_t &smem)
 {
     const int T = a.T, T_pad = (T + 15) / 16 * 16, W = (T + 31) / 32;
     const int hpt = a.P >= RB ? 1 : RB / a.P;
     const int NB = RB / 64, KA = (T_pad + 63) / 64;
     p.dt_box = a.H < kDtBox ? a.H : kDtBox;
-    uint32_t off = 2u * RB * 512u;                            // h0 stages
+    uint32_t off = (uint32_t)S * RB * 512u;                   // h0 stages
     p.off_x = off;
     p.x_dt = (uint32_t)NB * T_pad * 128u;
     p.x_stage = round_up(p.x_dt + (uint32_t)T * p.dt_box * 2u, 1024u);
-    off += 2u * p.x_stage;
+    off += (uint32_t)S * p.x_stage;
     // MMA rows past the tile (h0 rows >= RB, the second x block when RB = 64)
     // read whatever follows; keep that inside the allocation.
     const uint32_t spill = (uint32_t)(128 - RB) * 128u > (uint32_t)T_pad * 128u ? (uint32_t)(128 - RB) * 128u
@@ -689,15 +768,17 @@ bool layout(const ScanArgs &a, int RB, TcParams &p, size_t &smem)
     p.off_pnode = round_up(off, 16u);  off = p.off_pnode + (uint32_t)T * 2u;
     p.off_bar = round_up(off, 16u);    off = p.off_bar + kNumBars * 8u;
     p.off_misc = round_up(off, 16u);   off = p.off_misc + kMiscWords * 4u;
+    p.off_ad = round_up(off, 16u);     off = p.off_ad + 2u * a.H * 4u;
     p.off_pcb = round_up(off, 16u);
     const size_t fixed = (size_t)p.off_pcb + 1024;            // + alignment slack of the dynamic base
-    if (fixed + 5 * 64 + 16 > kSmemLimit) return false;
+    if (fixed + 6 * 64 + 32 > kSmemLimit) return false;
     const int all_pairs = T * (T + 1) / 2;
-    int cap = (int)((kSmemLimit - fixed - 16) / 5);
+    int cap = (int)((kSmemLimit - fixed - 32) / 6);
     if (cap > all_pairs) cap = all_pairs;
     p.pair_cap = cap;
     p.off_pj = round_up(p.off_pcb + (uint32_t)cap * 4u, 16u);
-    smem = (size_t)p.off_pj + cap + 1024;
+    p.off_pi = round_up(p.off_pj + (uint32_t)cap, 16u);
+    smem = (size_t)p.off_pi + cap + 1024;
     smem = (smem + 15) / 16 * 16;
     if (smem > kSmemLimit) return false;
     p.T = T;
@@ -705,6 +786,7 @@ bool layout(const ScanArgs &a, int RB, TcParams &p, size_t &smem)
     p.KA = KA;
     p.RB = RB;
     p.NB = NB;
+    p.S = S;
     p.hpt = hpt;
     p.acc_cols = (1 + hpt) * T_pad;
     uint32_t cols = 32;
@@ -725,24 +807,37 @@ bool rb_valid(const ScanArgs &a, int RB)
 bool plan(const ScanArgs &a, TcPlan &pl)
 {
     if (a.dtype != STREE_BF16 || a.N != kDstate || a.T > kMaxTcNodes || a.P % 32 != 0 || a.H % 8 != 0) return false;
-    if (a.batch <= 0 || a.H % a.G != 0) return false;
+    if (a.batch <= 0 || a.H % a.G != 0 || a.H > kMaxSmemHeads) return false;
     if (!encode_fn()) return false;
     const int sms = num_sms();
+    // Preference: three stages (loads two tiles ahead), then the tallest tile
+    // that still gives every SM work.
+    const int cand[4][2] = {{128, 3}, {64, 3}, {128, 2}, {64, 2}};
     int chosen = -1;
+    long long chosen_tiles = -1;
     TcParams best{};
     size_t best_smem = 0;
-    for (int RB : {128, 64}) {
+    for (const auto &c : cand) {
+        const int RB = c[0], S = c[1];
         TcParams p{};
         size_t smem = 0;
-        if (!rb_valid(a, RB) || !layout(a, RB, p, smem)) continue;
-        // Room for the ancestor pairs of typical trees (about 4 per node).
-        if (p.pair_cap < 4 * a.T && p.pair_cap < a.T * (a.T + 1) / 2 && RB > 64) continue;
+        if (!rb_valid(a, RB) || !layout(a, RB, S, p, smem)) continue;
+        const int all_pairs = a.T * (a.T + 1) / 2;
+        if (p.pair_cap < all_pairs && p.pair_cap < 4 * a.T) continue;   // typical trees must fit
         const long long ntiles = (long long)a.batch * (a.H * a.P / RB);
         if (ntiles > 0x7fffffff) continue;
-        chosen = RB;
-        best = p;
-        best_smem = smem;
-        if (ntiles >= sms) break;                  // largest tile that still fills the GPU
+        if (ntiles >= sms) {
+            chosen = RB;
+            best = p;
+            best_smem = smem;
+            break;
+        }
+        if (ntiles > chosen_tiles) {
+            chosen = RB;
+            chosen_tiles = ntiles;
+            best = p;
+            best_smem = smem;
+        }
     }
     if (chosen < 0) return false;
     best.H = a.H;
