@@ -229,6 +229,19 @@ __device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, con
     }
 }
 
+#ifdef STREE_TRACE
+// Profiling builds only: wall-clock stamps of pipeline events for four CTAs.
+__device__ unsigned long long g_trace[4 * 32 * 16];
+__device__ __forceinline__ void trace_event(uint32_t k, int ev)
+{
+    const int slot = blockIdx.x == 0 ? 0 : blockIdx.x == 37 ? 1 : blockIdx.x == 74 ? 2 : blockIdx.x == 111 ? 3 : -1;
+    if (slot >= 0 && k < 32) g_trace[(slot * 32 + k) * 16 + ev] = ptx::globaltimer();
+}
+#define STREE_TR(k, ev) trace_event((k), (ev))
+#else
+#define STREE_TR(k, ev) ((void)0)
+#endif
+
 __device__ __forceinline__ void named_sync(int id, int nthreads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -343,6 +356,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         }
         ptx::bulk_commit();
         stores_issued = q + 1;
+        STREE_TR(q, 10);
     };
     // Producer: TMA loads of tile k into stage k % S once tile k - S has left it.
     auto produce = [&](uint32_t k, int t) {
@@ -350,6 +364,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         if (k >= (uint32_t)S) {
             store_tile(k - S);
             ptx::bulk_wait_read_all();
+            STREE_TR(k - S, 11);
         }
         if (misc[M_ABORT]) return;
         const int b = t / p.tps, r0 = (t % p.tps) * RB;
@@ -362,6 +377,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         for (int nb = 0; nb < p.NB; ++nb) ptx::tma_load_2d(xdst + nb * xbs, &tm_x, r0 + nb * 64, b * T, fb);
         ptx::tma_load_2d(xdst + p.x_dt, &tm_dt, hf8, b * T, fb);
         loads_issued = k + 1;
+        STREE_TR(k, 0);
     };
 
     int cur_key = -1, cur_b = -1;
@@ -386,6 +402,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 produced = true;
             }
             __syncthreads();                                   // every earlier tile is consumed
+            if (tid == 0) STREE_TR(k, 12);
             const bool new_b = (b != cur_b);
             // Phase 1: independent loads.
             for (int q = tid; q < T_pad * 32; q += kThreads) {
@@ -500,6 +517,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             ptx::fence_proxy_async_smem();
             __syncthreads();
+            if (tid == 0) STREE_TR(k, 13);
             cur_key = key;
         }
         const int len = misc[M_LEN];
@@ -517,6 +535,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 const uint32_t acc = tmem + (uint32_t)(a * p.acc_cols);
                 bool ok = wait(bar(B_FULL + s), sph, 20);
                 if (ok && k >= 2) ok = wait(bar(B_ACCE + a), ((k >> 1) - 1) & 1, 21);
+                STREE_TR(k, 1);
                 if (ok) {
                     ptx::tc_fence_after();
                     const uint32_t a0 = ptx::smem_u32(h0t), b0 = ptx::smem_u32(cs);
@@ -529,6 +548,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                                           ptx::desc_kmajor_sw128(b0 + kb * T_pad * 128 + kk * 32), idesc_root,
                                           (kb | kk) != 0);
                     ok = wait(bar(B_MHF), k & 1, 22);
+                    STREE_TR(k, 2);
                 }
                 if (ok) {
                     ptx::tc_fence_after();
@@ -544,6 +564,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     ptx::mma_commit(bar(B_ACCF + a));
                     ptx::mma_commit(bar(B_MHE));
+                    STREE_TR(k, 3);
                 }
             }
         } else if (warp < kEpiWarp0) {
@@ -554,6 +575,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             if (ok && k >= 2) ok = wait(bar(B_COEFE + c), ((k >> 1) - 1) & 1, 31);
             float *dts = coef(c, 0), *Ls = coef(c, 1), *eLs = coef(c, 2), *wts = coef(c, 3);
             float *alpha = coef(c, 4);
+            if (ptid == 0) STREE_TR(k, 4);
             if (ok) {
                 const __nv_bfloat16 *dtt = reinterpret_cast<const __nv_bfloat16 *>(xt + p.x_dt);
                 const int hoff = hfirst - (hfirst & ~7);
@@ -592,6 +614,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     if (ptid < hpt) alpha[ptid] = len > 0 ? eLs[ptid * T + leaf] : 1.f;
                 }
                 mbar_arrive(bar(B_COEFF + c));
+                if (ptid == 0) STREE_TR(k, 5);
                 // Masked decay matrix of every head of the tile (bf16, K-major swizzled):
                 // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i.
                 ok = (k == 0) || wait(bar(B_MHE), (k - 1) & 1, 32);
@@ -618,6 +641,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     ptx::fence_proxy_async_smem();
                     mbar_arrive(bar(B_MHF));
+                    if (ptid == 0) STREE_TR(k, 6);
                 }
             }
         } else {
@@ -630,6 +654,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             named_sync(kBarEpi, kEpiThreads);
             // Warp-uniform decision: tcgen05.ld below is a warp-collective instruction.
             const bool run = __all_sync(0xffffffffu, ok && !misc[M_ABORT]);
+            if (etid == 0) STREE_TR(k, 7);
             if (run) ptx::tc_fence_after();
             const float *eLs = coef(c, 2), *wts = coef(c, 3), *alpha = coef(c, 4);
             if (run && commit) {
@@ -642,6 +667,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     commit_rows<32>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, c_lo);
             }
             named_sync(kBarEpi, kEpiThreads);                  // x rows of the path are read
+            if (etid == 0) STREE_TR(k, 8);
             // A warp reads only its own quarter of the tensor-memory lanes: 32 * (warp % 4).
             const int quad = warp & 3, half = ewarp >> 2;
             if (run && quad * 32 < RB) {
@@ -674,6 +700,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             ptx::fence_proxy_async_smem();
             named_sync(kBarEpi, kEpiThreads);
+            if (etid == 0) STREE_TR(k, 9);
             if (run && etid == 0) {
                 misc[M_SDESC + 2 * s] = t;                     // the producer issues the stores
                 misc[M_SDESC + 2 * s + 1] = commit ? 1 : 0;
@@ -933,3 +960,15 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
 }
 
 }  // namespace stree
+
+#ifdef STREE_TRACE
+extern "C" int stree_debug_trace(unsigned long long *host, size_t n)
+{
+    return (int)cudaMemcpyFromSymbol(host, stree::g_trace, n * sizeof(unsigned long long));
+}
+extern "C" int stree_debug_trace_clear(void)
+{
+    static unsigned long long zero[4 * 32 * 16];
+    return (int)cudaMemcpyToSymbol(stree::g_trace, zero, sizeof(zero));
+}
+#endif
