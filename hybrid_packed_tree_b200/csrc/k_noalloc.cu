@@ -1,0 +1,129 @@
+// k_noalloc.cu -- the fused scan + commit for callers that must not allocate.
+//
+// Some callers cannot call cudaMalloc at the point where they run the scan: a
+// serving runtime that owns all device memory through its own pool and forbids
+// stray allocations, code running under a memory cap that is already reached,
+// or a hot loop whose allocator calls would synchronise the device.  This entry
+// point runs the same kernels as stree_tree_scan_commit, but takes its scratch
+// (tree masks, depths, per-sequence flags, the C.B pair scratch of the CUDA-core
+// kernel and, when the caller gives none, the error word) from one file-scope
+// device array instead of a context's workspace.
+//
+// That array is a static __device__ object: every GPU that loads the library
+// holds its kNoAllocScratch bytes until the process exits.  Host code may not
+// pass the array's name to a kernel -- on the host it is only a stand-in -- so
+// the device address is looked up with cudaGetSymbolAddress, once per device,
+// with that device current, on the first call made on it.
+#include <mutex>
+#include <string.h>
+
+#include "stree_internal.cuh"
+
+namespace stree {
+namespace {
+
+constexpr size_t kNoAllocScratch = size_t(8) << 20;   // 8 MiB per device
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratch];
+
+std::mutex g_mutex;
+uint8_t *g_scratch[kMaxDevices] = {};
+
+// Device address of the scratch on the current device (looked up once per device).
+cudaError_t scratch_address(uint8_t **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_scratch[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch[dev] = static_cast<uint8_t *>(p);
+    }
+    *out = g_scratch[dev];
+    return cudaSuccess;
+}
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace stree
+
+using namespace stree;
+
+extern "C" stree_status stree_tree_scan_commit_noalloc(
+    const void *x, const void *dt, const float *A, const void *B, const void *C, const float *D, const float *h0,
+    const int32_t *parent, int n_nodes, int batch, int nheads, int headdim, int dstate, int ngroups,
+    stree_dtype dtype, const int32_t *accepted_path, const int32_t *path_len, int maxlen, void *y, float *h_new,
+    int32_t *err_out, void *stream)
+{
+    ScanArgs a{};
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.h0 = h0;
+    a.T = n_nodes; a.batch = batch; a.H = nheads; a.P = headdim; a.N = dstate; a.G = ngroups;
+    a.dtype = dtype;
+    a.y = y;
+    a.path = accepted_path;
+    a.path_len = path_len;
+    a.maxlen = maxlen;
+    a.h_new = h_new;
+
+    // Same shape rules as the context entry points.
+    if (batch < 0 || n_nodes < 1 || nheads < 1 || ngroups < 1 || headdim < 1 || dstate < 1) return STREE_ERR_UNSUPPORTED;
+    if (n_nodes > kMaxNodes || headdim > kMaxDim || dstate > kMaxDim) return STREE_ERR_UNSUPPORTED;
+    if (headdim % 8 != 0 || dstate % 8 != 0 || nheads % ngroups != 0 || nheads > 65535) return STREE_ERR_UNSUPPORTED;
+    if (dtype != STREE_F32 && dtype != STREE_BF16) return STREE_ERR_UNSUPPORTED;
+    if (maxlen < 1) return STREE_ERR_INVALID_ARG;
+    if (batch == 0) return STREE_OK;
+    if (!x || !dt || !A || !B || !C || !D || !h0 || !y || !parent || !accepted_path || !path_len || !h_new)
+        return STREE_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, dt, A, B, C, D, h0, y, h_new};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return STREE_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(parent) & 3u) || (reinterpret_cast<uintptr_t>(accepted_path) & 3u) ||
+        (reinterpret_cast<uintptr_t>(path_len) & 3u) || (reinterpret_cast<uintptr_t>(err_out) & 3u))
+        return STREE_ERR_MISALIGNED;
+
+    // Scratch layout: error word, masks, depths, flags, then the C.B pair
+    // scratch when the CUDA-core kernel runs.  Sizes beyond the array are rejected.
+    const size_t T = (size_t)n_nodes, W = (T + 31) / 32, nb = (size_t)batch;
+    const size_t off_err = 0;
+    const size_t off_anc = 256;
+    const size_t off_depth = off_anc + round256(nb * T * W * sizeof(uint32_t));
+    const size_t off_ok = off_depth + round256(nb * T * sizeof(int32_t));
+    const size_t off_cb = off_ok + round256(nb * sizeof(int32_t));
+    if (off_cb > kNoAllocScratch) return STREE_ERR_UNSUPPORTED;
+    // The tensor-core path's plan needs the device; look the scratch up first.
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *base = nullptr;
+    if (scratch_address(&base) != cudaSuccess) return STREE_ERR_CUDA;
+    const bool use_tc = tc_supported(a);
+    size_t need = off_cb;
+    if (!use_tc) need += round256(nb * (size_t)ngroups * T * T * sizeof(float));
+    if (need > kNoAllocScratch) return STREE_ERR_UNSUPPORTED;
+
+    int32_t *err = err_out ? err_out : reinterpret_cast<int32_t *>(base + off_err);
+    uint32_t *anc = reinterpret_cast<uint32_t *>(base + off_anc);
+    int32_t *depth = reinterpret_cast<int32_t *>(base + off_depth);
+    int32_t *ok = reinterpret_cast<int32_t *>(base + off_ok);
+    // The error word must start at zero; masks, depths, flags and the pair
+    // scratch are fully rewritten by the kernels below.
+    if (cudaMemsetAsync(err, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return STREE_ERR_CUDA;
+    if (launch_build_tree(parent, n_nodes, batch, anc, depth, ok, err, s) != cudaSuccess) return STREE_ERR_CUDA;
+    a.tree.anc = anc;
+    a.tree.depth = depth;
+    a.tree.ok = ok;
+    a.tree.T = n_nodes;
+    a.tree.W = (int)W;
+    a.tree.batch = batch;
+    a.err = err;
+    if (use_tc) return launch_scan_tc(a, s) == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
+    a.cb = reinterpret_cast<float *>(base + off_cb);
+    if (launch_cb_pairs(a, s) != cudaSuccess) return STREE_ERR_CUDA;
+    return launch_scan_simt(a, s) == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
+}

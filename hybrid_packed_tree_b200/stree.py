@@ -38,7 +38,8 @@ KERNELS = {"auto": 0, "simt": 1, "tc": 2}
 EXPORTS = (
     "stree_ctx_create", "stree_ctx_destroy", "stree_ctx_set_kernel", "stree_ctx_launch_count",
     "stree_build_tree",
-    "stree_tree_scan", "stree_commit", "stree_tree_scan_commit", "stree_resolve_path",
+    "stree_tree_scan", "stree_commit", "stree_tree_scan_commit", "stree_tree_scan_commit_noalloc",
+    "stree_resolve_path",
     "stree_sync_check", "stree_status_string", "stree_version",
 )
 
@@ -51,6 +52,7 @@ _lib.stree_build_tree.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp]
 _lib.stree_tree_scan.argtypes = [_vp] * 9 + [_i] * 7 + [_vp, _vp]
 _lib.stree_commit.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
 _lib.stree_tree_scan_commit.argtypes = [_vp] * 9 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp]
+_lib.stree_tree_scan_commit_noalloc.argtypes = [_vp] * 8 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp, _vp]
 _lib.stree_resolve_path.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
 _lib.stree_sync_check.argtypes = [_vp, _vp, _ip]
 _lib.stree_status_string.argtypes = [_i]
@@ -201,6 +203,23 @@ def stree_tree_scan_commit(ctx: Ctx, x, dt, A, B, C, D, h0, parent, path, path_l
                                      _ptr(path_len, "path_len", (torch.int32,)), path.shape[1],
                                      yp, _ptr(h_new, "h_new", (torch.float32,)), _stream(stream))
     _check(st, "stree_tree_scan_commit")
+    return y, h_new
+
+
+def stree_tree_scan_commit_noalloc(x, dt, A, B, C, D, h0, parent, path, path_len, y, h_new, err_out=None,
+                                   stream=None):
+    """(y, h_new) <- fused scan + commit with no context and no allocation.
+
+    Scratch comes from the library's fixed device array; err_out (device int32[4])
+    receives this call's error word.  Calls on one device must not overlap.
+    """
+    ins, yp = _scan_ptrs(x, dt, A, B, C, D, h0, y)
+    st = _lib.stree_tree_scan_commit_noalloc(*ins, _ptr(parent, "parent", (torch.int32,)), *_dims(x, B),
+                                             _io_dtype(x), _ptr(path, "path", (torch.int32,)),
+                                             _ptr(path_len, "path_len", (torch.int32,)), path.shape[1], yp,
+                                             _ptr(h_new, "h_new", (torch.float32,)),
+                                             _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
+    _check(st, "stree_tree_scan_commit_noalloc")
     return y, h_new
 
 

@@ -147,6 +147,32 @@ stree_status stree_tree_scan_commit(stree_ctx *ctx, const void *x, const void *d
                                     int maxlen, void *y, float *h_new, void *stream);
 
 /*
+ * Fused scan + commit that allocates nothing (the paper has no counterpart:
+ * this is a deployment convenience).  For callers that may not allocate device
+ * memory where they run the scan -- a serving runtime that hands out all device
+ * memory from its own pool, a process already at its memory cap, or a hot loop
+ * where an allocator call would synchronise the device.  Arguments are those of
+ * stree_tree_scan_commit without the context, plus err_out: a device int32[4]
+ * that receives the error word of this call ({status, sequence, position,
+ * detail}; cleared by the call), or NULL to discard device-detected errors.
+ *
+ * Scratch: the tree masks, depths and flags (and the CUDA-core kernel's C.B
+ * pair scratch) live in one file-scope device array of 8 MiB that every GPU
+ * loading the library keeps until the process exits.  Sizes whose scratch does
+ * not fit return STREE_ERR_UNSUPPORTED before anything is launched.  The first
+ * call on a device looks the array's device address up (cudaGetSymbolAddress);
+ * make that first call before any stream capture.  Every call on a device
+ * shares the array, so calls that overlap on the GPU (other streams, other host
+ * threads) race; serialise them.  The call never calls cudaMalloc or cudaFree.
+ */
+stree_status stree_tree_scan_commit_noalloc(const void *x, const void *dt, const float *A, const void *B,
+                                            const void *C, const float *D, const float *h0, const int32_t *parent,
+                                            int n_nodes, int batch, int nheads, int headdim, int dstate,
+                                            int ngroups, stree_dtype dtype, const int32_t *accepted_path,
+                                            const int32_t *path_len, int maxlen, void *y, float *h_new,
+                                            int32_t *err_out, void *stream);
+
+/*
  * Resolve accepted paths against the context's current tree: leaf_out[b] (device
  * int32 [batch]) receives the last node of a valid path, -1 for an empty path and
  * -2 for an invalid one (which also latches STREE_ERR_BAD_PATH).

@@ -103,4 +103,14 @@ def test_binding_argtypes_match_header(lib_path):
         if name.startswith("stree_") and fn.argtypes and name not in (
                 "stree_status_string", "stree_ctx_create", "stree_ctx_destroy"):
             args = [0 if t is ctypes.c_int else None for t in fn.argtypes]
-            assert fn(*args) == 1, name
+            # NULL context / zero sizes: rejected on the host before any device work.
+            assert fn(*args) in (1, 2), name
+
+
+def test_noalloc_rejects_oversized_scratch_on_the_host(lib_path):
+    """Sizes whose tree scratch exceeds the fixed 8 MiB array fail before any device call."""
+    from hybrid_packed_tree_b200 import stree
+    fn = stree._lib.stree_tree_scan_commit_noalloc
+    fake = 0x10000                                    # aligned, never dereferenced
+    args = [fake] * 8 + [256, 1 << 16, 8, 64, 128, 1, 1] + [fake, fake, 256, fake, fake, None, None]
+    assert fn(*args) == 2
