@@ -172,9 +172,9 @@ struct MnCol {
     }
 };
 
-// Commit of one tile row segment: h_new = alpha h0 + sum_q coef_q B[pnode_q] (fp32).
-// The first kPathRows path rows of B come from shared memory (fp32), later ones
-// from global memory.
+// Commit of one tile row segment: h_new = alpha h0 + sum_q coef_q B[pnode_q] (fp32),
+// coef_q = w_q x[pnode_q][row].  The first kPathRows path rows of B come from shared
+// memory (fp32, fully unrolled), later ones from global memory.
 template <int CPT>
 __device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, const MnCol &xc, const float *Bp,
                                             const __nv_bfloat16 *Bseq, size_t brow, const int16_t *pnode,
@@ -183,64 +183,126 @@ __device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, con
     float acc[CPT];
 #pragma unroll
     for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
-    for (int q = 0; q < len; ++q) {
-        const int j = pnode[q];
-        const float coef = wh[q] * bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
-        if (q < kPathRows) {
+    float cf[kPathRows];
+#pragma unroll
+    for (int q = 0; q < kPathRows; ++q) {
+        // Only path positions q < len hold node indices; others address node 0.
+        const int j = q < len ? (int)pnode[q] : 0;
+        const float xv = bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
+        cf[q] = q < len ? wh[q] * xv : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < kPathRows; ++q) {
+        if (q < len) {
             const float4 *src = reinterpret_cast<const float4 *>(Bp + q * kDstate + c_lo);
 #pragma unroll
             for (int c = 0; c < CPT / 4; ++c) {
                 const float4 bv = src[c];
-                acc[4 * c + 0] = fmaf(coef, bv.x, acc[4 * c + 0]);
-                acc[4 * c + 1] = fmaf(coef, bv.y, acc[4 * c + 1]);
-                acc[4 * c + 2] = fmaf(coef, bv.z, acc[4 * c + 2]);
-                acc[4 * c + 3] = fmaf(coef, bv.w, acc[4 * c + 3]);
-            }
-        } else {
-            const uint2 *src = reinterpret_cast<const uint2 *>(Bseq + (size_t)j * brow + c_lo);
-#pragma unroll
-            for (int c = 0; c < CPT / 4; ++c) {
-                float b0, b1, b2, b3;
-                unpack4(__ldg(src + c), b0, b1, b2, b3);
-                acc[4 * c + 0] = fmaf(coef, b0, acc[4 * c + 0]);
-                acc[4 * c + 1] = fmaf(coef, b1, acc[4 * c + 1]);
-                acc[4 * c + 2] = fmaf(coef, b2, acc[4 * c + 2]);
-                acc[4 * c + 3] = fmaf(coef, b3, acc[4 * c + 3]);
+                acc[4 * c + 0] = fmaf(cf[q], bv.x, acc[4 * c + 0]);
+                acc[4 * c + 1] = fmaf(cf[q], bv.y, acc[4 * c + 1]);
+                acc[4 * c + 2] = fmaf(cf[q], bv.z, acc[4 * c + 2]);
+                acc[4 * c + 3] = fmaf(cf[q], bv.w, acc[4 * c + 3]);
             }
         }
     }
-    float4 h[CPT / 4];
+    for (int q = kPathRows; q < len; ++q) {
+        const int j = pnode[q];
+        const float coef = wh[q] * bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
+        const uint2 *src = reinterpret_cast<const uint2 *>(Bseq + (size_t)j * brow + c_lo);
 #pragma unroll
-    for (int c = 0; c < CPT / 4; ++c) {
-        const int n = c_lo + 4 * c;
-        const int kb = n >> 5, ch = (n & 31) >> 2;
-        h[c] = *reinterpret_cast<const float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
+        for (int c = 0; c < CPT / 4; ++c) {
+            float b0, b1, b2, b3;
+            unpack4(__ldg(src + c), b0, b1, b2, b3);
+            acc[4 * c + 0] = fmaf(coef, b0, acc[4 * c + 0]);
+            acc[4 * c + 1] = fmaf(coef, b1, acc[4 * c + 1]);
+            acc[4 * c + 2] = fmaf(coef, b2, acc[4 * c + 2]);
+            acc[4 * c + 3] = fmaf(coef, b3, acc[4 * c + 3]);
+        }
     }
 #pragma unroll
-    for (int c = 0; c < CPT / 4; ++c) {
-        const int n = c_lo + 4 * c;
-        const int kb = n >> 5, ch = (n & 31) >> 2;
-        float4 v;
-        v.x = fmaf(al, h[c].x, acc[4 * c + 0]);
-        v.y = fmaf(al, h[c].y, acc[4 * c + 1]);
-        v.z = fmaf(al, h[c].z, acc[4 * c + 2]);
-        v.w = fmaf(al, h[c].w, acc[4 * c + 3]);
-        *reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+    for (int c0 = 0; c0 < CPT / 4; c0 += 4) {
+        float4 h[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int n = c_lo + 4 * (c0 + c);
+            const int kb = n >> 5, ch = (n & 31) >> 2;
+            h[c] = *reinterpret_cast<const float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4));
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int n = c_lo + 4 * (c0 + c);
+            const int kb = n >> 5, ch = (n & 31) >> 2;
+            float4 v;
+            v.x = fmaf(al, h[c].x, acc[4 * (c0 + c) + 0]);
+            v.y = fmaf(al, h[c].y, acc[4 * (c0 + c) + 1]);
+            v.z = fmaf(al, h[c].z, acc[4 * (c0 + c) + 2]);
+            v.w = fmaf(al, h[c].w, acc[4 * (c0 + c) + 3]);
+            *reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+        }
     }
 }
 
 #ifdef STREE_TRACE
 // Profiling builds only: wall-clock stamps of pipeline events for four CTAs.
-__device__ unsigned long long g_trace[4 * 32 * 16];
+__device__ unsigned long long g_trace[4 * 32 * 24];
 __device__ __forceinline__ void trace_event(uint32_t k, int ev)
 {
     const int slot = blockIdx.x == 0 ? 0 : blockIdx.x == 37 ? 1 : blockIdx.x == 74 ? 2 : blockIdx.x == 111 ? 3 : -1;
-    if (slot >= 0 && k < 32) g_trace[(slot * 32 + k) * 16 + ev] = ptx::globaltimer();
+    if (slot >= 0 && k < 32) g_trace[(slot * 32 + k) * 24 + ev] = ptx::globaltimer();
 }
 #define STREE_TR(k, ev) trace_event((k), (ev))
 #else
 #define STREE_TR(k, ev) ((void)0)
 #endif
+
+// Eight 16-bit shared-memory loads issued back to back (addresses in the shared window).
+__device__ __forceinline__ void lds_u16x8(const uint32_t (&a)[8], uint16_t (&v)[8])
+{
+    asm volatile(
+        "ld.shared.u16 %0, [%8];\n\t"
+        "ld.shared.u16 %1, [%9];\n\t"
+        "ld.shared.u16 %2, [%10];\n\t"
+        "ld.shared.u16 %3, [%11];\n\t"
+        "ld.shared.u16 %4, [%12];\n\t"
+        "ld.shared.u16 %5, [%13];\n\t"
+        "ld.shared.u16 %6, [%14];\n\t"
+        "ld.shared.u16 %7, [%15];"
+        : "=h"(v[0]), "=h"(v[1]), "=h"(v[2]), "=h"(v[3]), "=h"(v[4]), "=h"(v[5]), "=h"(v[6]), "=h"(v[7])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void lds_f32x8(const uint32_t (&a)[8], float (&v)[8])
+{
+    asm volatile(
+        "ld.shared.f32 %0, [%8];\n\t"
+        "ld.shared.f32 %1, [%9];\n\t"
+        "ld.shared.f32 %2, [%10];\n\t"
+        "ld.shared.f32 %3, [%11];\n\t"
+        "ld.shared.f32 %4, [%12];\n\t"
+        "ld.shared.f32 %5, [%13];\n\t"
+        "ld.shared.f32 %6, [%14];\n\t"
+        "ld.shared.f32 %7, [%15];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void sts_u16x8(const uint32_t (&a)[8], const uint16_t (&v)[8])
+{
+    asm volatile(
+        "st.shared.u16 [%0], %8;\n\t"
+        "st.shared.u16 [%1], %9;\n\t"
+        "st.shared.u16 [%2], %10;\n\t"
+        "st.shared.u16 [%3], %11;\n\t"
+        "st.shared.u16 [%4], %12;\n\t"
+        "st.shared.u16 [%5], %13;\n\t"
+        "st.shared.u16 [%6], %14;\n\t"
+        "st.shared.u16 [%7], %15;"
+        :: "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]),
+           "h"(v[0]), "h"(v[1]), "h"(v[2]), "h"(v[3]), "h"(v[4]), "h"(v[5]), "h"(v[6]), "h"(v[7])
+        : "memory");
+}
 
 __device__ __forceinline__ void named_sync(int id, int nthreads)
 {
@@ -257,8 +319,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
                const __grid_constant__ CUtensorMap tm_dt, const TcParams p)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base.  Offsetting the __shared__ array itself (rather than
+    // rounding an integer address) keeps every derived pointer in the shared state
+    // space, so accesses compile to shared-memory instructions, not generic ones.
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = p.T, T_pad = p.T_pad, RB = p.RB, P = p.P, H = p.H, G = p.G, W = p.tree.W, HP = H * P;
     const int hpg = H / G, hpt = p.hpt, S = p.S;
@@ -539,7 +604,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 if (ok) {
                     ptx::tc_fence_after();
                     const uint32_t a0 = ptx::smem_u32(h0t), b0 = ptx::smem_u32(cs);
-                    const uint32_t idesc_root = ptx::idesc_tf32(128, T_pad);
+                    const uint32_t idesc_root = ptx::idesc_tf32(RB, T_pad);
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
@@ -553,7 +618,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 if (ok) {
                     ptx::tc_fence_after();
                     const uint32_t xa = ptx::smem_u32(xt);
-                    const uint32_t idesc_tree = ptx::idesc_bf16_amn(128, T_pad);
+                    const uint32_t idesc_tree = ptx::idesc_bf16_amn(RB, T_pad);
                     for (int hh = 0; hh < hpt; ++hh) {
                         const uint32_t mb = ptx::smem_u32(mh + hh * p.mh_head);
                         const uint32_t dcol = acc + (uint32_t)(T_pad * (1 + hh));
@@ -571,8 +636,13 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             // ------------------------------------------------------------ prep warps
             const int ptid = tid - kPrepWarp0 * 32;
             const int c = k & 1;
-            bool ok = wait(bar(B_FULL + s), sph, 30);
-            if (ok && k >= 2) ok = wait(bar(B_COEFE + c), ((k >> 1) - 1) & 1, 31);
+            // One thread polls the barriers; the others sleep on the named barrier.
+            if (ptid == 0) {
+                bool w = wait(bar(B_FULL + s), sph, 30);
+                if (w && k >= 2) w = wait(bar(B_COEFE + c), ((k >> 1) - 1) & 1, 31);
+            }
+            named_sync(kBarPrep, kPrepThreads);
+            bool ok = !misc[M_ABORT];
             float *dts = coef(c, 0), *Ls = coef(c, 1), *eLs = coef(c, 2), *wts = coef(c, 3);
             float *alpha = coef(c, 4);
             if (ptid == 0) STREE_TR(k, 4);
@@ -617,7 +687,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 if (ptid == 0) STREE_TR(k, 5);
                 // Masked decay matrix of every head of the tile (bf16, K-major swizzled):
                 // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i.
-                ok = (k == 0) || wait(bar(B_MHE), (k - 1) & 1, 32);
+                if (ptid == 0 && k > 0) wait(bar(B_MHE), (k - 1) & 1, 32);
+                named_sync(kBarPrep, kPrepThreads);
+                ok = !misc[M_ABORT];
                 if (ok) {
                     const int total = misc[M_TOTAL];
                     if (misc[M_INSMEM]) {
@@ -648,12 +720,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             // ------------------------------------------------------------ epilogue warps
             const int etid = tid - kEpiWarp0 * 32, ewarp = warp - kEpiWarp0;
             const int a = k & 1, c = k & 1;
-            bool ok = wait(bar(B_FULL + s), sph, 40);
-            if (ok) ok = wait(bar(B_COEFF + c), (k >> 1) & 1, 41);
-            if (ok) ok = wait(bar(B_ACCF + a), (k >> 1) & 1, 42);
+            // One thread polls the barriers; the others sleep on the named barrier.
+            if (etid == 0) {
+                bool w = wait(bar(B_FULL + s), sph, 40);
+                if (w) w = wait(bar(B_COEFF + c), (k >> 1) & 1, 41);
+                if (w) w = wait(bar(B_ACCF + a), (k >> 1) & 1, 42);
+            }
             named_sync(kBarEpi, kEpiThreads);
-            // Warp-uniform decision: tcgen05.ld below is a warp-collective instruction.
-            const bool run = __all_sync(0xffffffffu, ok && !misc[M_ABORT]);
+            // Warp-uniform decision (tcgen05.ld below is a warp-collective instruction).
+            const bool run = __all_sync(0xffffffffu, !misc[M_ABORT]);
             if (etid == 0) STREE_TR(k, 7);
             if (run) ptx::tc_fence_after();
             const float *eLs = coef(c, 2), *wts = coef(c, 3), *alpha = coef(c, 4);
@@ -666,32 +741,79 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 for (int c_lo = part * cols; c_lo < (part + 1) * cols; c_lo += 32)
                     commit_rows<32>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, c_lo);
             }
+            if (warp == 8 && lane == 0) STREE_TR(k, 19);
             named_sync(kBarEpi, kEpiThreads);                  // x rows of the path are read
             if (etid == 0) STREE_TR(k, 8);
             // A warp reads only its own quarter of the tensor-memory lanes: 32 * (warp % 4).
+            // M = 128 puts tile row r in lane r; M = 64 puts rows 16q..16q+15 in
+            // lanes 32q..32q+15, so every quarter (and every SM sub-partition) gets rows.
             const int quad = warp & 3, half = ewarp >> 2;
-            if (run && quad * 32 < RB) {
-                const int row = quad * 32 + lane;
+            // With M = 64 lanes 16..31 of a quarter hold no rows: those threads load
+            // (tcgen05.ld is warp-collective) but do not store.
+            const bool active = RB == 128 || lane < 16;
+            const int row = RB == 128 ? quad * 32 + lane : quad * 16 + (lane & 15);
+            if (run) {
                 const int hh = (r0 + row) / P - hfirst;           // same for the whole warp (P >= 32)
                 const float Dh = Dsh[hfirst + hh];
                 const float *eLh = eLs + hh * T;
                 const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * p.acc_cols);
                 const uint32_t ty = tl + (uint32_t)(T_pad * (1 + hh));
                 const MnCol xc(row, xbs);
-                for (int c0 = half * 16; c0 < T; c0 += 32) {
-                    float R[16], Y[16], X[16];
-                    ptx::tmem_ld16(tl + (uint32_t)c0, R);
-                    ptx::tmem_ld16(ty + (uint32_t)c0, Y);
+                const uint32_t xbase = ptx::smem_u32(xt), ebase = ptx::smem_u32(eLh);
+                // Chunks of 8 nodes; the next chunk's tensor-memory values are loaded
+                // while the current one is computed.
+                uint32_t R[8], Y[8], Rn[8], Yn[8];
+                int c0 = half * 8;
+                if (c0 < T) {
+                    ptx::tmem_ld8_nowait(tl + (uint32_t)c0, R);
+                    ptx::tmem_ld8_nowait(ty + (uint32_t)c0, Y);
+                    ptx::tmem_wait_ld();
+                }
+                for (; c0 < T; c0 += 16) {
+                    const bool more = c0 + 16 < T;
+                    if (more) {
+                        ptx::tmem_ld8_nowait(tl + (uint32_t)(c0 + 16), Rn);
+                        ptx::tmem_ld8_nowait(ty + (uint32_t)(c0 + 16), Yn);
+                    }
+                    // Nodes past T read row T-1 and their results are dropped (every
+                    // address stays inside the stage).
+                    uint32_t xa[8], ea[8];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        X[u] = (c0 + u < T) ? bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(c0 + u))) : 0.f;
+                    for (int u = 0; u < 8; ++u) {
+                        const int i = min(c0 + u, T - 1);
+                        xa[u] = xbase + xc.at(i);
+                        ea[u] = ebase + (uint32_t)i * 4u;
+                    }
+                    uint16_t Xh[8];
+                    float E[8];
+                    lds_u16x8(xa, Xh);
+                    lds_f32x8(ea, E);
+                    uint16_t Yh[8];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        if (c0 + u < T)
-                            *reinterpret_cast<__nv_bfloat16 *>(xt + xc.at(c0 + u)) =
-                                __float2bfloat16_rn(fmaf(eLh[c0 + u], R[u], fmaf(Dh, X[u], Y[u])));
+                    for (int u = 0; u < 8; ++u) {
+                        const float xv = __uint_as_float((uint32_t)Xh[u] << 16);
+                        const float yv = fmaf(E[u], __uint_as_float(R[u]), fmaf(Dh, xv, __uint_as_float(Y[u])));
+                        Yh[u] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
+                    }
+                    if (active && c0 + 8 <= T) {
+                        sts_u16x8(xa, Yh);
+                    } else if (active) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            if (c0 + u < T)
+                                asm volatile("st.shared.u16 [%0], %1;" ::"r"(xa[u]), "h"(Yh[u]) : "memory");
+                    }
+                    if (more) {
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            R[u] = Rn[u];
+                            Y[u] = Yn[u];
+                        }
+                    }
                 }
             }
+            if (warp == 8 && lane == 0) STREE_TR(k, 16);
             ptx::tc_fence_before();
             __syncwarp();
             if (run && lane == 0) {
@@ -699,6 +821,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 mbar_arrive(bar(B_COEFE + c));
             }
             ptx::fence_proxy_async_smem();
+            if (warp == 8 && lane == 0) STREE_TR(k, 17);
+            if (warp == 6 && lane == 0) STREE_TR(k, 18);
             named_sync(kBarEpi, kEpiThreads);
             if (etid == 0) STREE_TR(k, 9);
             if (run && etid == 0) {
@@ -968,7 +1092,7 @@ extern "C" int stree_debug_trace(unsigned long long *host, size_t n)
 }
 extern "C" int stree_debug_trace_clear(void)
 {
-    static unsigned long long zero[4 * 32 * 16];
+    static unsigned long long zero[4 * 32 * 24];
     return (int)cudaMemcpyToSymbol(stree::g_trace, zero, sizeof(zero));
 }
 #endif
