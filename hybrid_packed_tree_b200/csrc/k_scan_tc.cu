@@ -963,7 +963,7 @@ bool plan(const ScanArgs &a, TcPlan &pl)
     const int sms = num_sms();
     // Preference: three stages (loads two tiles ahead), then the tallest tile
     // that still gives every SM work.
-    const int cand[4][2] = {{128, 3}, {64, 3}, {128, 2}, {64, 2}};
+    const int cand[4][2] = {{128, 3}, {128, 2}, {64, 3}, {64, 2}};
     int chosen = -1;
     long long chosen_tiles = -1;
     TcParams best{};
