@@ -42,7 +42,6 @@ namespace {
 
 constexpr int kDstate = 128;               // dstate of the tensor-core path
 constexpr int kMaxTcNodes = 128;           // T_pad <= 128 (TMEM columns, smem)
-constexpr int kDtBox = 16;                 // heads per dt box (32 bytes of bf16)
 constexpr int kPathRows = 8;               // accepted-path rows of B staged in smem (fp32)
 constexpr size_t kSmemLimit = 232448;      // 227 KB opt-in dynamic shared memory
 
@@ -63,6 +62,7 @@ enum Bars { B_FULL = 0, B_EPID = kMaxStages, B_ACCF = 2 * kMaxStages, B_ACCE = B
             B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, kNumBars = B_COEFE + 2 };
 
 struct TcParams {
+    const __nv_bfloat16 *__restrict__ dt;
     const __nv_bfloat16 *__restrict__ B;
     const __nv_bfloat16 *__restrict__ C;
     const float *__restrict__ A;
@@ -71,9 +71,9 @@ struct TcParams {
     const int32_t *__restrict__ path_len;
     TreeView tree;
     int32_t *err;
-    int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, hpt, pair_cap, dt_box, acc_cols;
+    int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, hpt, pair_cap, acc_cols;
     uint32_t tmem_cols;
-    uint32_t off_x, x_dt, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_coef, coef_slot,
+    uint32_t off_x, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_coef, coef_slot,
         off_pnode, off_bar, off_misc, off_ad, off_pcb, off_pj, off_pi;
 };
 
@@ -317,7 +317,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
 __global__ void __launch_bounds__(kThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant__ CUtensorMap tm_hn,
                const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
-               const __grid_constant__ CUtensorMap tm_dt, const TcParams p)
+               const TcParams p)
 {
     // 1024-byte aligned base.  Offsetting the __shared__ array itself (rather than
     // rounding an integer address) keeps every derived pointer in the shared state
@@ -351,12 +351,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     auto bar = [&](int i) { return ptx::smem_u32(&bars[i]); };
 
     const uint32_t h0_stage_bytes = (uint32_t)RB * 512u;
-    const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u + (uint32_t)T * p.dt_box * 2u;
+    const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u;
 
     if (tid == 0) {
         ptx::prefetch_tensormap(&tm_h0);
         ptx::prefetch_tensormap(&tm_x);
-        ptx::prefetch_tensormap(&tm_dt);
         ptx::prefetch_tensormap(&tm_hn);
         ptx::prefetch_tensormap(&tm_y);
         for (int s = 0; s < kMaxStages; ++s) {
@@ -417,7 +416,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         for (int nb = 0; nb < p.NB; ++nb) ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
         if (commit) {
             const uint32_t src = ptx::smem_u32(h0s + s * h0_stage_bytes);
-            for (int kb = 0; kb < 4; ++kb) ptx::tma_store_2d(&tm_hn, kb * 32, b * HP + r0, src + kb * RB * 128);
+            ptx::tma_store_3d(&tm_hn, 0, b * HP + r0, 0, src);
         }
         ptx::bulk_commit();
         stores_issued = q + 1;
@@ -433,14 +432,12 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         }
         if (misc[M_ABORT]) return;
         const int b = t / p.tps, r0 = (t % p.tps) * RB;
-        const int hf8 = (r0 / P) & ~7;
         const uint32_t fb = bar(B_FULL + s);
         ptx::mbar_expect_tx(fb, tx_bytes);
         const uint32_t dst = ptx::smem_u32(h0s + s * h0_stage_bytes);
-        for (int kb = 0; kb < 4; ++kb) ptx::tma_load_2d(dst + kb * RB * 128, &tm_h0, kb * 32, b * HP + r0, fb);
+        ptx::tma_load_3d(dst, &tm_h0, 0, b * HP + r0, 0, fb);    // [4 column groups][RB rows][32]
         const uint32_t xdst = ptx::smem_u32(xs + s * p.x_stage);
         for (int nb = 0; nb < p.NB; ++nb) ptx::tma_load_2d(xdst + nb * xbs, &tm_x, r0 + nb * 64, b * T, fb);
-        ptx::tma_load_2d(xdst + p.x_dt, &tm_dt, hf8, b * T, fb);
         loads_issued = k + 1;
         STREE_TR(k, 0);
     };
@@ -636,22 +633,19 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             // ------------------------------------------------------------ prep warps
             const int ptid = tid - kPrepWarp0 * 32;
             const int c = k & 1;
-            // One thread polls the barriers; the others sleep on the named barrier.
-            if (ptid == 0) {
-                bool w = wait(bar(B_FULL + s), sph, 30);
-                if (w && k >= 2) w = wait(bar(B_COEFE + c), ((k >> 1) - 1) & 1, 31);
-            }
+            // Prep needs only dt, A and the topology -- not the tile's TMA stage -- so
+            // it runs ahead of the load.  One thread polls; the others sleep on the
+            // named barrier.
+            if (ptid == 0 && k >= 2) wait(bar(B_COEFE + c), ((k >> 1) - 1) & 1, 31);
             named_sync(kBarPrep, kPrepThreads);
             bool ok = !misc[M_ABORT];
             float *dts = coef(c, 0), *Ls = coef(c, 1), *eLs = coef(c, 2), *wts = coef(c, 3);
             float *alpha = coef(c, 4);
             if (ptid == 0) STREE_TR(k, 4);
             if (ok) {
-                const __nv_bfloat16 *dtt = reinterpret_cast<const __nv_bfloat16 *>(xt + p.x_dt);
-                const int hoff = hfirst - (hfirst & ~7);
                 for (int q = ptid; q < hpt * T; q += kPrepThreads) {
                     const int hh = q / T, i = q - hh * T;
-                    dts[q] = bf2f(dtt[i * p.dt_box + hoff + hh]);
+                    dts[q] = bf2f(p.dt[((size_t)b * T + i) * H + hfirst + hh]);
                 }
             }
             named_sync(kBarPrep, kPrepThreads);
@@ -895,11 +889,9 @@ bool layout(const ScanArgs &a, int RB, int S, TcParams &p, size_t &smem)
     const int T = a.T, T_pad = (T + 15) / 16 * 16, W = (T + 31) / 32;
     const int hpt = a.P >= RB ? 1 : RB / a.P;
     const int NB = RB / 64, KA = (T_pad + 63) / 64;
-    p.dt_box = a.H < kDtBox ? a.H : kDtBox;
     uint32_t off = (uint32_t)S * RB * 512u;                   // h0 stages
     p.off_x = off;
-    p.x_dt = (uint32_t)NB * T_pad * 128u;
-    p.x_stage = round_up(p.x_dt + (uint32_t)T * p.dt_box * 2u, 1024u);
+    p.x_stage = round_up((uint32_t)NB * T_pad * 128u, 1024u);
     off += (uint32_t)S * p.x_stage;
     // MMA rows past the tile (h0 rows >= RB, the second x block when RB = 64)
     // read whatever follows; keep that inside the allocation.
@@ -957,7 +949,7 @@ bool rb_valid(const ScanArgs &a, int RB)
 
 bool plan(const ScanArgs &a, TcPlan &pl)
 {
-    if (a.dtype != STREE_BF16 || a.N != kDstate || a.T > kMaxTcNodes || a.P % 32 != 0 || a.H % 8 != 0) return false;
+    if (a.dtype != STREE_BF16 || a.N != kDstate || a.T > kMaxTcNodes || a.P % 32 != 0) return false;
     if (a.batch <= 0 || a.H % a.G != 0 || a.H > kMaxSmemHeads) return false;
     if (!encode_fn()) return false;
     const int sms = num_sms();
@@ -1014,6 +1006,7 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     TcPlan pl;
     if (!plan(a, pl)) return cudaErrorNotSupported;
     TcParams p = pl.p;
+    p.dt = static_cast<const __nv_bfloat16 *>(a.dt);
     p.B = static_cast<const __nv_bfloat16 *>(a.B);
     p.C = static_cast<const __nv_bfloat16 *>(a.C);
     p.A = a.A;
@@ -1027,18 +1020,20 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
 
     EncodeTiledFn enc = encode_fn();
     const int HP = a.H * a.P;
-    CUtensorMap m_h0, m_hn, m_x, m_y, m_dt;
+    CUtensorMap m_h0, m_hn, m_x, m_y;
     {
-        cuuint64_t dims[2] = {(cuuint64_t)kDstate, (cuuint64_t)a.batch * HP};
-        cuuint64_t strides[1] = {(cuuint64_t)kDstate * 4};
-        cuuint32_t box[2] = {32, (cuuint32_t)p.RB};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&m_h0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(a.h0), dims, strides, box, es,
+        // h0 / h_new as [4 groups of 32 columns][rows][32 columns]: one box is a
+        // whole tile in the K-major layout of the MMA (four 128-byte-swizzled atoms).
+        cuuint64_t dims[3] = {32, (cuuint64_t)a.batch * HP, kDstate / 32};
+        cuuint64_t strides[2] = {(cuuint64_t)kDstate * 4, 128};
+        cuuint32_t box[3] = {32, (cuuint32_t)p.RB, kDstate / 32};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&m_h0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(a.h0), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
         float *hn = p.do_commit ? a.h_new : const_cast<float *>(a.h0);
-        if (enc(&m_hn, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, hn, dims, strides, box, es,
+        if (enc(&m_hn, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, hn, dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
@@ -1057,16 +1052,6 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    {
-        cuuint64_t dims[2] = {(cuuint64_t)a.H, (cuuint64_t)a.batch * a.T};
-        cuuint64_t strides[1] = {(cuuint64_t)a.H * 2};
-        cuuint32_t box[2] = {(cuuint32_t)p.dt_box, (cuuint32_t)a.T};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&m_dt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.dt), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
     cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
     if (e != cudaSuccess) return e;
     cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -1079,7 +1064,7 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     if (per_sm > tmem_fit) per_sm = tmem_fit;
     long long grid = (long long)num_sms() * per_sm;
     if (grid > p.ntiles) grid = p.ntiles;
-    scan_tc_kernel<<<(unsigned)grid, kThreads, pl.smem, s>>>(m_h0, m_hn, m_x, m_y, m_dt, p);
+    scan_tc_kernel<<<(unsigned)grid, kThreads, pl.smem, s>>>(m_h0, m_hn, m_x, m_y, p);
     return cudaGetLastError();
 }
 
