@@ -402,6 +402,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         return false;
     };
 
+    // Launched as a programmatic dependent of the tree builder: everything above
+    // overlapped it; the tree masks, depths and flags are read only after this.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     const int start = (int)((long long)blockIdx.x * p.ntiles / gridDim.x);
     const int end = (int)((long long)(blockIdx.x + 1) * p.ntiles / gridDim.x);
     uint32_t loads_issued = 0, stores_issued = 0;
@@ -1064,8 +1068,19 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     if (per_sm > tmem_fit) per_sm = tmem_fit;
     long long grid = (long long)num_sms() * per_sm;
     if (grid > p.ntiles) grid = p.ntiles;
-    scan_tc_kernel<<<(unsigned)grid, kThreads, pl.smem, s>>>(m_h0, m_hn, m_x, m_y, p);
-    return cudaGetLastError();
+    // Programmatic dependent launch: the prologue (barriers, tensor memory, A/D)
+    // overlaps the preceding kernel, normally the tree builder.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, scan_tc_kernel, m_h0, m_hn, m_x, m_y, p);
 }
 
 }  // namespace stree

@@ -21,6 +21,9 @@ __global__ void __launch_bounds__(256) build_tree_kernel(const int32_t *__restri
     __shared__ uint32_t rows[kMaxNodes * kMaxWords];
     __shared__ int bad;
     const int b = blockIdx.x;
+    // A scan launched as a programmatic dependent may start its prologue now; it
+    // waits for this grid's completion before it reads the masks.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) bad = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < T; i += blockDim.x) {
