@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample budget")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--layers", type=int, default=None, help="override the workload's layer count (profiling)")
+    ap.add_argument("--also", default="serve64",
+                    help="comma-separated extra workloads summarised in the same line ('none' to skip)")
     return ap.parse_args()
 
 
@@ -84,27 +86,29 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic(kernel_name):
-    """Per-launch DRAM bytes of the dominant kernel from the committed ncu summary,
-    if that summary was taken on the current kernel source; else None."""
+def source_sha(fname):
     import hashlib
+    src = os.path.join(ROOT, "hybrid_packed_tree_b200", "csrc", fname)
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else None
+
+
+def profile_traffic(kernel_name, workload):
+    """Per-launch DRAM bytes (read + write) of the dominant kernel for this workload,
+    from the committed ncu summary, if it was taken on the current kernel source;
+    else None."""
     summ = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(summ):
         return None
-    want = None
     for line in open(summ):
-        if line.startswith("traffic:"):
-            kv = dict(t.split("=", 1) for t in line[len("traffic:"):].split())
-            want = kv
-    if not want or want.get("kernel") != kernel_name:
-        return None
-    src = os.path.join(ROOT, "hybrid_packed_tree_b200", "csrc", want.get("file", ""))
-    if not os.path.exists(src):
-        return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if sha != want.get("sha"):
-        return None
-    return float(want["bytes_per_launch"])
+        if not line.startswith("traffic:"):
+            continue
+        kv = dict(t.split("=", 1) for t in line[len("traffic:"):].split())
+        if kv.get("kernel") != kernel_name or kv.get("workload") != workload:
+            continue
+        if source_sha(kv.get("file", "")) != kv.get("sha"):
+            return None
+        return float(kv["bytes_per_launch"])
+    return None
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -157,6 +161,25 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- ranks
+
+
+def max_over_ranks(values, world, device):
+    """Each timing becomes its maximum over the ranks (identity on one rank)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_scaling_value(units_per_rank_step, steps, ms, world):
+    """Whole-job throughput: every rank processes its own batch, time is the slowest rank's."""
+    return world * units_per_rank_step * steps / (ms / 1e3)
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -261,15 +284,10 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device error during the benchmark: {info}")
 
-    if world > 1:
-        t = torch.tensor([ms, statistics.mean(kern_ms)], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, kmean = float(t[0]), float(t[1])
-    else:
-        kmean = statistics.mean(kern_ms)
+    ms, kmean = max_over_ranks([ms, statistics.mean(kern_ms)], world, device)
 
     nodes_step = w.batch * w.n_nodes * nl
-    value = world * nodes_step * K / (ms / 1e3)
+    value = weak_scaling_value(nodes_step, K, ms, world)
     hbm_gbs, peak_kind = peaks()
     achieved = launch_bytes / (kmean / 1e3) / 1e9
     kernel_name = "scan_tc_kernel" if args.kernel != "simt" else "scan_simt_kernel"
@@ -288,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
         "sequences_per_s": world * w.batch * K / (ms / 1e3),
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
-            "frac": achieved / hbm_gbs, "traffic": profile_traffic(kernel_name),
+            "frac": achieved / hbm_gbs, "traffic": profile_traffic(kernel_name, args.config),
             "peak_source": f"{peak_kind} hbm_gbs", "kernel": kernel_name,
             "bytes_per_launch": launch_bytes, "kernel_ms_mean": kmean,
             "kernel_ms_median": statistics.median(kern_ms),
@@ -350,12 +368,9 @@ def e2e(torch, stree, w, ctx, device, stream, args, world):
     t1.record(stream)
     torch.cuda.synchronize(device)
     ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+    (ms,) = max_over_ranks([ms], world, device)
     nodes = w.batch * w.n_nodes * w.nlayers
-    return {"value": world * nodes * K / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+    return {"value": weak_scaling_value(nodes, K, ms, world), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": K}
 
 
@@ -443,6 +458,21 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     out = run_ours(args, rank, world, local_rank)
+    extras = [] if args.also in ("", "none") else [c for c in args.also.split(",") if c and c != args.config]
+    if extras:
+        import copy
+        out["other_workloads"] = {}
+        for name in extras:
+            a2 = copy.copy(args)
+            a2.config, a2.no_e2e, a2.steps, a2.batch, a2.layers = name, True, None, None, None
+            o2 = run_ours(a2, rank, world, local_rank)
+            r2 = o2["roofline"]
+            out["other_workloads"][name] = {
+                "value": o2["value"], "unit": o2["unit"], "ms_per_step": o2["ms_per_step"], "steps": o2["steps"],
+                "config": o2["config"], "clocks": o2["clocks"],
+                "roofline": {k: r2[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic",
+                                                "bytes_per_launch", "kernel_ms_mean")},
+            }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_seconds)
     if rank == 0:
