@@ -121,6 +121,7 @@ extern "C" stree_status stree_tree_scan_commit_noalloc(
     a.tree.T = n_nodes;
     a.tree.W = (int)W;
     a.tree.batch = batch;
+    a.parent = parent;                       // the builder was launched right before
     a.err = err;
     if (use_tc) return launch_scan_tc(a, s) == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
     a.cb = reinterpret_cast<float *>(base + off_cb);

@@ -11,25 +11,29 @@
 // Design (B200).  The state h0 [b, H*P, N=128] streams through the SMs in tiles
 // of RB rows of the flattened (head, headdim) axis; a persistent CTA walks a
 // contiguous range of tiles with warp-specialised roles joined by mbarriers:
-//   * producer warp: TMA loads of the fp32 h0 tile (128-byte swizzled, 4 boxes
-//     of 32 columns), the bf16 x tile (64-column swizzled boxes) and the dt box
-//     into a 2-stage ring;
+//   * producer warp: TMA loads of the fp32 h0 tile (one 3-D box: four 128-byte
+//     swizzled atoms of 32 columns) and the bf16 x tile (64-column swizzled
+//     boxes) into an S-stage ring (S = 2 or 3), and the TMA stores of y and h_new;
 //   * MMA warp (one thread): the root term R[row, i] = h0[row, :] . C_i as
 //     tcgen05.mma kind::tf32 (M = 128, N = T_pad, K = 128) and the tree term
 //     Y[row, i] = sum_j x[j, row] M_h[i, j] as kind::f16 with x as an MN-major
 //     operand straight from the stage, into a 2-deep tensor-memory ring;
 //   * prep warps: per tile and head the tree cumsum L, exp(L) and the masked
 //     decay matrix M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j over ancestor
-//     pairs only (bf16, K-major swizzled), plus the commit weights;
+//     pairs only, with D_h added on the diagonal (bf16, K-major swizzled), plus
+//     the commit weights;
 //   * epilogue warps: the commit in exact fp32 FMA, written in place over the
-//     h0 tile, then y = exp(L_i) R + Y + D x in place over the x tile, then TMA
-//     stores of both and the release of the stage.
+//     h0 tile, then y = exp(L_i) R + Y in place over the x tile (Y already holds
+//     the skip term), and the release of the stage to the producer's stores.
 // C (fp32 operand of the root MMA), the ancestor pairs' C.B and the accepted
-// path's rows of B are staged once per (sequence, group).  Roles only block on
+// path's rows of B are staged once per (sequence, group), all of its global
+// reads issued together.  When the call passes parent[] the kernel builds the
+// tree masks itself in shared memory and requests its first tiles at entry, so
+// it never waits for the tree builder launched beside it.  Roles only block on
 // bounded mbarrier waits; a timeout latches STREE_ERR_TIMEOUT and the CTA runs
 // to its end without further work.  Precision: the root term rounds h0 to tf32
-// and the masked decay matrix to bf16 inside the MMAs (fp32 accumulation); the
-// commit and every other step are fp32.
+// and the masked decay matrix (D_h on its diagonal included) to bf16 inside the
+// MMAs (fp32 accumulation); the commit and every other step are fp32.
 #include <cuda.h>
 
 #include <mutex>
@@ -53,13 +57,15 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kPrepThreads = kPrepWarps * 32, kEpiThreads = kEpiWarps * 32;
 constexpr int kBarEpi = 1, kBarPrep = 2;   // named barriers (0 is __syncthreads)
 
-enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_SDESC = 8, M_WSUM = 8 + 2 * kMaxStages,
+enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_OK, M_DTK, M_SDESC = 8, M_WSUM = 8 + 2 * kMaxStages,
             kMiscWords = M_WSUM + kWarps };
 // mbarriers: TMA stage full / epilogue done with a stage (ring of S), tensor-memory
-// accumulator full / empty (ring of 2), masked-decay matrix full / empty, and
-// per-tile coefficients full / empty (ring of 2).
+// accumulator full / empty (ring of 2), masked-decay matrix full / empty,
+// per-tile coefficients full / empty (ring of 2), and for the tensor-core commit
+// its coefficient operand ready / its product done.
 enum Bars { B_FULL = 0, B_EPID = kMaxStages, B_ACCF = 2 * kMaxStages, B_ACCE = B_ACCF + 2, B_MHF = B_ACCE + 2,
-            B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, kNumBars = B_COEFE + 2 };
+            B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, B_CFF = B_COEFE + 2, B_CMF = B_CFF + 1,
+            kNumBars = B_CMF + 1 };
 
 struct TcParams {
     const __nv_bfloat16 *__restrict__ dt;
@@ -69,12 +75,15 @@ struct TcParams {
     const float *__restrict__ D;
     const int32_t *__restrict__ path;
     const int32_t *__restrict__ path_len;
+    const int32_t *__restrict__ parent;    // non-NULL: masks built in-kernel, inputs complete at launch
     TreeView tree;
     int32_t *err;
-    int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, hpt, pair_cap, acc_cols;
+    int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, pre, bs_mh, tc_commit, hpt, pair_cap,
+        acc_cols, cm_col;
     uint32_t tmem_cols;
     uint32_t off_x, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_coef, coef_slot,
-        off_pnode, off_bar, off_misc, off_ad, off_pcb, off_pj, off_pi;
+        off_pnode, off_praw, off_par, off_dep, off_bs, off_cf, off_bt, off_bar, off_misc, off_ad, off_pcb, off_pj,
+        off_pi;
 };
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -130,7 +139,9 @@ __device__ __forceinline__ float dot_cb(const uint8_t *cs, int T_pad, const __nv
 }
 
 // C_i . B_j over the quarter `part` (32 of the 128 state columns); four lanes of
-// a warp combine their parts with shuffles.
+// a warp combine their parts with shuffles.  B_j is read from shared memory
+// (kStaged) or from global memory.
+template <bool kStaged>
 __device__ __forceinline__ float dot_cb_part(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i, int part)
 {
     float acc = 0.f;
@@ -138,7 +149,7 @@ __device__ __forceinline__ float dot_cb_part(const uint8_t *cs, int T_pad, const
     const uint2 *brow = reinterpret_cast<const uint2 *>(Bj) + part * 8;
     uint2 raw[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) raw[c] = __ldg(brow + c);
+    for (int c = 0; c < 8; ++c) raw[c] = kStaged ? brow[c] : __ldg(brow + c);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const float4 cv = *reinterpret_cast<const float4 *>(crow + ((c ^ (i & 7)) << 4));
@@ -172,53 +183,66 @@ struct MnCol {
     }
 };
 
-// Commit of one tile row segment: h_new = alpha h0 + sum_q coef_q B[pnode_q] (fp32),
-// coef_q = w_q x[pnode_q][row].  The first kPathRows path rows of B come from shared
-// memory (fp32, fully unrolled), later ones from global memory.
+// Two fp32 fused multiply-adds in one instruction (lane-wise a * b + c, each
+// rounded once, exactly as two scalar fmaf).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const unsigned long long *>(&a)), "l"(*reinterpret_cast<const unsigned long long *>(&b)),
+          "l"(*reinterpret_cast<const unsigned long long *>(&c)));
+    return *reinterpret_cast<float2 *>(&d);
+}
+
+// Commit of one tile row segment on CUDA cores: h_new = alpha h0 + sum_q coef_q B[pnode_q]
+// (fp32), coef_q = w_q x[pnode_q][row], written in place over the h0 tile.  The
+// first `nsm` (<= kPathRows) path rows of B come from shared memory (fp32), the
+// others from global memory.
 template <int CPT>
-__device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, const MnCol &xc, const float *Bp,
+__device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, const MnCol &xc, const float *Bp, int nsm,
                                             const __nv_bfloat16 *Bseq, size_t brow, const int16_t *pnode,
                                             const float *wh, float al, int len, int RB, int row, int c_lo)
 {
-    float acc[CPT];
+    float2 acc[CPT / 2];
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
+    for (int c = 0; c < CPT / 2; ++c) acc[c] = make_float2(0.f, 0.f);
+    const int lsm = min(len, nsm);
     float cf[kPathRows];
 #pragma unroll
     for (int q = 0; q < kPathRows; ++q) {
-        // Only path positions q < len hold node indices; others address node 0.
-        const int j = q < len ? (int)pnode[q] : 0;
+        // Only path positions q < lsm are used here; others address node 0.
+        const int j = q < lsm ? (int)pnode[q] : 0;
         const float xv = bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
-        cf[q] = q < len ? wh[q] * xv : 0.f;
+        cf[q] = q < lsm ? wh[q] * xv : 0.f;
     }
 #pragma unroll
     for (int q = 0; q < kPathRows; ++q) {
-        if (q < len) {
+        if (q < lsm) {
             const float4 *src = reinterpret_cast<const float4 *>(Bp + q * kDstate + c_lo);
+            const float2 cq = make_float2(cf[q], cf[q]);
 #pragma unroll
             for (int c = 0; c < CPT / 4; ++c) {
                 const float4 bv = src[c];
-                acc[4 * c + 0] = fmaf(cf[q], bv.x, acc[4 * c + 0]);
-                acc[4 * c + 1] = fmaf(cf[q], bv.y, acc[4 * c + 1]);
-                acc[4 * c + 2] = fmaf(cf[q], bv.z, acc[4 * c + 2]);
-                acc[4 * c + 3] = fmaf(cf[q], bv.w, acc[4 * c + 3]);
+                acc[2 * c + 0] = ffma2(cq, make_float2(bv.x, bv.y), acc[2 * c + 0]);
+                acc[2 * c + 1] = ffma2(cq, make_float2(bv.z, bv.w), acc[2 * c + 1]);
             }
         }
     }
-    for (int q = kPathRows; q < len; ++q) {
+    for (int q = lsm; q < len; ++q) {
         const int j = pnode[q];
         const float coef = wh[q] * bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
+        const float2 cq = make_float2(coef, coef);
         const uint2 *src = reinterpret_cast<const uint2 *>(Bseq + (size_t)j * brow + c_lo);
 #pragma unroll
         for (int c = 0; c < CPT / 4; ++c) {
             float b0, b1, b2, b3;
             unpack4(__ldg(src + c), b0, b1, b2, b3);
-            acc[4 * c + 0] = fmaf(coef, b0, acc[4 * c + 0]);
-            acc[4 * c + 1] = fmaf(coef, b1, acc[4 * c + 1]);
-            acc[4 * c + 2] = fmaf(coef, b2, acc[4 * c + 2]);
-            acc[4 * c + 3] = fmaf(coef, b3, acc[4 * c + 3]);
+            acc[2 * c + 0] = ffma2(cq, make_float2(b0, b1), acc[2 * c + 0]);
+            acc[2 * c + 1] = ffma2(cq, make_float2(b2, b3), acc[2 * c + 1]);
         }
     }
+    const float2 a2 = make_float2(al, al);
 #pragma unroll
     for (int c0 = 0; c0 < CPT / 4; c0 += 4) {
         float4 h[4];
@@ -232,14 +256,20 @@ __device__ __forceinline__ void commit_rows(uint8_t *h0t, const uint8_t *xt, con
         for (int c = 0; c < 4; ++c) {
             const int n = c_lo + 4 * (c0 + c);
             const int kb = n >> 5, ch = (n & 31) >> 2;
-            float4 v;
-            v.x = fmaf(al, h[c].x, acc[4 * (c0 + c) + 0]);
-            v.y = fmaf(al, h[c].y, acc[4 * (c0 + c) + 1]);
-            v.z = fmaf(al, h[c].z, acc[4 * (c0 + c) + 2]);
-            v.w = fmaf(al, h[c].w, acc[4 * (c0 + c) + 3]);
-            *reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+            const float2 lo = ffma2(a2, make_float2(h[c].x, h[c].y), acc[2 * (c0 + c) + 0]);
+            const float2 hi = ffma2(a2, make_float2(h[c].z, h[c].w), acc[2 * (c0 + c) + 1]);
+            *reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 + ((ch ^ (row & 7)) << 4)) =
+                make_float4(lo.x, lo.y, hi.x, hi.y);
         }
     }
+}
+
+// Byte offset of fp32 element (row, k), k < 8, in a K-major operand without
+// swizzle: 8-row x 16-byte core matrices of 128 contiguous bytes, the two
+// K-halves of a row group 128 bytes apart, row groups 256 bytes apart.
+__device__ __forceinline__ uint32_t k8_off(int row, int k)
+{
+    return (uint32_t)(row >> 3) * 256u + (uint32_t)(k >> 2) * 128u + (uint32_t)(row & 7) * 16u + (uint32_t)(k & 3) * 4u;
 }
 
 #ifdef STREE_TRACE
@@ -255,23 +285,7 @@ __device__ __forceinline__ void trace_event(uint32_t k, int ev)
 #define STREE_TR(k, ev) ((void)0)
 #endif
 
-// Eight 16-bit shared-memory loads issued back to back (addresses in the shared window).
-__device__ __forceinline__ void lds_u16x8(const uint32_t (&a)[8], uint16_t (&v)[8])
-{
-    asm volatile(
-        "ld.shared.u16 %0, [%8];\n\t"
-        "ld.shared.u16 %1, [%9];\n\t"
-        "ld.shared.u16 %2, [%10];\n\t"
-        "ld.shared.u16 %3, [%11];\n\t"
-        "ld.shared.u16 %4, [%12];\n\t"
-        "ld.shared.u16 %5, [%13];\n\t"
-        "ld.shared.u16 %6, [%14];\n\t"
-        "ld.shared.u16 %7, [%15];"
-        : "=h"(v[0]), "=h"(v[1]), "=h"(v[2]), "=h"(v[3]), "=h"(v[4]), "=h"(v[5]), "=h"(v[6]), "=h"(v[7])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7])
-        : "memory");
-}
-
+// Eight 32-bit shared-memory loads issued back to back (addresses in the shared window).
 __device__ __forceinline__ void lds_f32x8(const uint32_t (&a)[8], float (&v)[8])
 {
     asm volatile(
@@ -325,18 +339,23 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int T = p.T, T_pad = p.T_pad, RB = p.RB, P = p.P, H = p.H, G = p.G, W = p.tree.W, HP = H * P;
+    const int T = p.T, T_pad = p.T_pad, RB = p.RB, P = p.P, H = p.H, G = p.G, HP = H * P;
+    const int W = (T + 31) / 32;
     const int hpg = H / G, hpt = p.hpt, S = p.S;
     const uint32_t xbs = (uint32_t)T_pad * 128u;                      // x: bytes per 64-column block
 
     uint8_t *h0s = smem;                                              // S x [4 atoms][RB rows][128 B] fp32
-    uint8_t *xs = smem + p.off_x;                                     // S x {NB x [T_pad rows][128 B] x, dt}
+    uint8_t *xs = smem + p.off_x;                                     // S x NB x [T_pad rows][128 B] bf16
     uint8_t *cs = smem + p.off_c;                                     // [4 atoms][T_pad rows][128 B] fp32
     uint8_t *mh = smem + p.off_mh;                                    // hpt x [KA atoms][T_pad rows][128 B] bf16
     float *Bp = reinterpret_cast<float *>(smem + p.off_bp);           // [kPathRows][128] fp32
     uint32_t *ancs = reinterpret_cast<uint32_t *>(smem + p.off_anc);  // [T][W]
     int32_t *poff = reinterpret_cast<int32_t *>(smem + p.off_poff);   // [T+1]
-    int16_t *pnode = reinterpret_cast<int16_t *>(smem + p.off_pnode); // [T]
+    int16_t *pnode = reinterpret_cast<int16_t *>(smem + p.off_pnode); // [T] validated accepted path
+    int32_t *praw = reinterpret_cast<int32_t *>(smem + p.off_praw);   // [T] accepted path as given
+    int32_t *par = reinterpret_cast<int32_t *>(smem + p.off_par);     // [T] parent as given
+    int32_t *dep = reinterpret_cast<int32_t *>(smem + p.off_dep);     // [T] depth
+    __nv_bfloat16 *Bs = reinterpret_cast<__nv_bfloat16 *>(smem + p.off_bs);   // [T][128] B rows, when staged
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     volatile int32_t *misc = reinterpret_cast<volatile int32_t *>(smem + p.off_misc);
     float *Ash = reinterpret_cast<float *>(smem + p.off_ad);          // [H] A, then [H] D
@@ -344,53 +363,25 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     float *pcb = reinterpret_cast<float *>(smem + p.off_pcb);         // [pair_cap] C_i . B_j
     uint8_t *pj = smem + p.off_pj;                                    // [pair_cap] j
     uint8_t *pi = smem + p.off_pi;                                    // [pair_cap] i
+    const bool b_staged = p.off_bs != 0;
+    uint8_t *cfs = smem + p.off_cf;                                   // [RB][8] fp32 commit coefficients (MMA A)
+    uint8_t *bts = smem + p.off_bt;                                   // [128][8] fp32 path rows of B^T (MMA B)
     // Per-tile coefficients, two slots: dts, L, exp(L), commit weights [hpt][T] each, alpha [hpt].
     auto coef = [&](int slot, int which) {
         return reinterpret_cast<float *>(smem + p.off_coef + slot * p.coef_slot) + which * hpt * T;
     };
     auto bar = [&](int i) { return ptx::smem_u32(&bars[i]); };
 
+    if (tid == 0) STREE_TR(31, 0);
     const uint32_t h0_stage_bytes = (uint32_t)RB * 512u;
     const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u;
-
-    if (tid == 0) {
-        ptx::prefetch_tensormap(&tm_h0);
-        ptx::prefetch_tensormap(&tm_x);
-        ptx::prefetch_tensormap(&tm_hn);
-        ptx::prefetch_tensormap(&tm_y);
-        for (int s = 0; s < kMaxStages; ++s) {
-            ptx::mbar_init(bar(B_FULL + s), 1);
-            ptx::mbar_init(bar(B_EPID + s), 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(bar(B_ACCF + s), 1);
-            ptx::mbar_init(bar(B_ACCE + s), kEpiWarps);
-            ptx::mbar_init(bar(B_COEFF + s), kPrepThreads);
-            ptx::mbar_init(bar(B_COEFE + s), kEpiWarps);
-        }
-        ptx::mbar_init(bar(B_MHF), kPrepThreads);
-        ptx::mbar_init(bar(B_MHE), 1);
-        ptx::fence_mbar_init();
-        for (int q = 0; q < kMiscWords; ++q) misc[q] = 0;
-    }
-    __syncthreads();                                  // misc cleared before the allocation writes it
-    // Operand rows the MMAs read past the valid tile (rows >= RB, nodes >= T)
-    // must hold finite values: clear the staging regions once.
-    for (uint32_t o = tid * 16u; o < p.off_mh; o += kThreads * 16u)
-        *reinterpret_cast<float4 *>(smem + o) = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int h = tid; h < H; h += kThreads) {
-        Ash[h] = __ldg(&p.A[h]);
-        Dsh[h] = __ldg(&p.D[h]);
-    }
-    if (warp == kMmaWarp) {
-        ptx::tmem_alloc(ptx::smem_u32(const_cast<int32_t *>(&misc[M_TMEM])), p.tmem_cols);
-        ptx::tmem_relinquish();
-    }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = static_cast<uint32_t>(misc[M_TMEM]);
+    const int start = (int)((long long)blockIdx.x * p.ntiles / gridDim.x);
+    const int end = (int)((long long)(blockIdx.x + 1) * p.ntiles / gridDim.x);
+    // With p.pre every input is complete at launch (the preceding launch is the
+    // tree builder, which started after all earlier work): the first S tiles are
+    // requested before anything else.
+    const uint32_t npre = p.pre ? (uint32_t)min(S, end - start) : 0u;
+    uint32_t loads_issued = 0, stores_issued = 0;
 
     // Bounded wait that turns a timeout into a CTA-wide abort; after an abort
     // every wait returns false at once and no role does further work.
@@ -401,27 +392,18 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         misc[M_ABORT] = 1;
         return false;
     };
-
-    // Launched as a programmatic dependent of the tree builder: everything above
-    // overlapped it; the tree masks, depths and flags are read only after this.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-
-    const int start = (int)((long long)blockIdx.x * p.ntiles / gridDim.x);
-    const int end = (int)((long long)(blockIdx.x + 1) * p.ntiles / gridDim.x);
-    uint32_t loads_issued = 0, stores_issued = 0;
-
-    // Producer: TMA stores of tile q once its epilogue is done (descriptor in misc).
+    // Producer: TMA stores of tile q once its epilogue is done (descriptor in misc:
+    // the tile, and bit 0 = store y, bit 1 = store h_new).
     auto store_tile = [&](uint32_t q) {
         const int s = q % S;
         if (!wait(bar(B_EPID + s), (q / S) & 1, 11)) return;
-        const int t = misc[M_SDESC + 2 * s], commit = misc[M_SDESC + 2 * s + 1];
+        const int t = misc[M_SDESC + 2 * s], what = misc[M_SDESC + 2 * s + 1];
         const int b = t / p.tps, r0 = (t % p.tps) * RB;
-        const uint32_t xsrc = ptx::smem_u32(xs + s * p.x_stage);
-        for (int nb = 0; nb < p.NB; ++nb) ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
-        if (commit) {
-            const uint32_t src = ptx::smem_u32(h0s + s * h0_stage_bytes);
-            ptx::tma_store_3d(&tm_hn, 0, b * HP + r0, 0, src);
+        if (what & 1) {
+            const uint32_t xsrc = ptx::smem_u32(xs + s * p.x_stage);
+            for (int nb = 0; nb < p.NB; ++nb) ptx::tma_store_2d(&tm_y, r0 + nb * 64, b * T, xsrc + nb * xbs);
         }
+        if (what & 2) ptx::tma_store_3d(&tm_hn, 0, b * HP + r0, 0, ptx::smem_u32(h0s + s * h0_stage_bytes));
         ptx::bulk_commit();
         stores_issued = q + 1;
         STREE_TR(q, 10);
@@ -446,11 +428,63 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         STREE_TR(k, 0);
     };
 
+    if (tid == 0) {
+        ptx::prefetch_tensormap(&tm_h0);
+        ptx::prefetch_tensormap(&tm_x);
+        ptx::prefetch_tensormap(&tm_hn);
+        ptx::prefetch_tensormap(&tm_y);
+        for (int s = 0; s < kMaxStages; ++s) {
+            ptx::mbar_init(bar(B_FULL + s), 1);
+            ptx::mbar_init(bar(B_EPID + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(bar(B_ACCF + s), 1);
+            ptx::mbar_init(bar(B_ACCE + s), kEpiWarps);
+            ptx::mbar_init(bar(B_COEFF + s), kPrepThreads);
+            ptx::mbar_init(bar(B_COEFE + s), kEpiWarps);
+        }
+        ptx::mbar_init(bar(B_MHF), kPrepThreads);
+        ptx::mbar_init(bar(B_MHE), 1);
+        ptx::mbar_init(bar(B_CFF), 1);
+        ptx::mbar_init(bar(B_CMF), 1);
+        ptx::fence_mbar_init();
+        for (int q = 0; q < kMiscWords; ++q) misc[q] = 0;
+        for (uint32_t q = 0; q < npre; ++q) produce(q, start + (int)q);
+    }
+    // x rows T..T_pad-1 of every stage are never written by the TMA but enter the
+    // tree MMA (times zero weights): keep them finite.  The TMA writes only rows < T.
+    {
+        const int padrows = T_pad - T, nchunks = S * p.NB * padrows * 8;
+        for (int q = tid; q < nchunks; q += kThreads) {
+            const int c16 = q & 7, r = (q >> 3) % padrows, blk = (q >> 3) / padrows;
+            uint8_t *dst = xs + (blk / p.NB) * p.x_stage + (blk % p.NB) * xbs + (T + r) * 128 + c16 * 16;
+            *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    // Without p.pre the inputs or the context's tree may come from the preceding
+    // launch: nothing global is read before it has completed.
+    if (!p.pre) asm volatile("griddepcontrol.wait;" ::: "memory");
+    __syncthreads();                                  // misc cleared before the allocation writes it
+    if (tid == 0) STREE_TR(31, 1);
+    if (warp == kMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_u32(const_cast<int32_t *>(&misc[M_TMEM])), p.tmem_cols);
+        ptx::tmem_relinquish();
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = static_cast<uint32_t>(misc[M_TMEM]);
+    if (tid == 0) STREE_TR(31, 2);
+
     int cur_key = -1, cur_b = -1;
+    // Prep warps: dt of the next tile, requested while the current one is prepared.
+    __nv_bfloat16 dnext[4];
+    int dnext_k = -1;
+    uint32_t ncm = 0;                                 // tiles committed on the tensor cores so far
     uint32_t k = 0;
-    for (int t = start; t < end; ++t) {
+    for (int t = start; t < end; ++t, ++k) {
         const int b = t / p.tps;
-        if (!__ldg(&p.tree.ok[b])) continue;                     // invalid tree: skipped by every role
         const int r0 = (t % p.tps) * RB;
         const int hfirst = r0 / P;
         const int g = hfirst / hpg;
@@ -459,59 +493,132 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         const uint32_t sph = (k / S) & 1;                        // phase parity of this stage use
         const __nv_bfloat16 *Bseq = p.B + ((size_t)b * T * G + g) * kDstate;   // row j at + j * G * 128
         const size_t brow = (size_t)G * kDstate;
-        bool produced = false;
+        bool produced = k < npre;
 
         // ------------------------------------------------------------ (sequence, group) switch
         if (key != cur_key) {
-            if (warp == kProducerWarp && lane == 0) {          // keep the stream going meanwhile
-                produce(k, t);
-                produced = true;
-            }
+            if (warp == kProducerWarp && lane == 0 && !produced) produce(k, t);   // keep the stream going
+            produced = true;
             __syncthreads();                                   // every earlier tile is consumed
             if (tid == 0) STREE_TR(k, 12);
             const bool new_b = (b != cur_b);
-            // Phase 1: independent loads.
-            for (int q = tid; q < T_pad * 32; q += kThreads) {
-                const int i = q >> 5, c = q & 31;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < T) {
-                    float c0, c1, c2, c3;
-                    unpack4(__ldg(reinterpret_cast<const uint2 *>(p.C + (((size_t)b * T + i) * G + g) * kDstate + c * 4)),
-                            c0, c1, c2, c3);
-                    v = make_float4(c0, c1, c2, c3);
+            // Phase 1: every global read of this (sequence, group) in flight at once:
+            // asynchronous copies for the B rows, parent, path, A and D (or the
+            // context's tree), plain loads for dt and C (C is widened to fp32).
+            if (b_staged)
+                for (int q = tid; q < T * 32; q += kThreads)
+                    ptx::cp_async8(ptx::smem_u32(Bs) + (uint32_t)q * 8u, Bseq + (size_t)(q >> 5) * brow + (q & 31) * 4);
+            if (cur_key < 0)
+                for (int h = tid; h < H; h += kThreads) {
+                    ptx::cp_async4(ptx::smem_u32(Ash + h), p.A + h);
+                    ptx::cp_async4(ptx::smem_u32(Dsh + h), p.D + h);
                 }
-                const int kb = c >> 3, ch = c & 7;
-                *reinterpret_cast<float4 *>(cs + kb * T_pad * 128 + i * 128 + ((ch ^ (i & 7)) << 4)) = v;
-            }
+            int plen = 0, okv = 1;
             if (new_b) {
-                for (int q = tid; q < T * W; q += kThreads) ancs[q] = __ldg(&p.tree.anc[(size_t)b * T * W + q]);
+                if (p.parent) {
+                    for (int i = tid; i < T; i += kThreads) ptx::cp_async4(ptx::smem_u32(par + i), p.parent + (size_t)b * T + i);
+                } else {
+                    for (int q = tid; q < T * W; q += kThreads)
+                        ptx::cp_async4(ptx::smem_u32(ancs + q), p.tree.anc + (size_t)b * T * W + q);
+                    for (int i = tid; i < T; i += kThreads) ptx::cp_async4(ptx::smem_u32(dep + i), p.tree.depth + (size_t)b * T + i);
+                    if (tid == 0) okv = __ldg(&p.tree.ok[b]);
+                }
+                if (p.do_commit) {
+                    for (int q = tid; q < min(p.maxlen, T); q += kThreads)
+                        ptx::cp_async4(ptx::smem_u32(praw + q), p.path + (size_t)b * p.maxlen + q);
+                    if (tid == 0) plen = __ldg(&p.path_len[b]);
+                }
+            }
+            // dt of this tile for the prep warps (hpt * T <= 512 values).
+            __nv_bfloat16 dtv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int q = tid + u * kThreads, hh = q / T, i = q - hh * T;
+                if (q < hpt * T) dtv[u] = p.dt[((size_t)b * T + i) * H + hfirst + hh];
+            }
+            {
+                // All of this thread's C loads are issued before the first is used.
+                constexpr int kCItems = (kMaxTcNodes * 32 + kThreads - 1) / kThreads;
+                uint2 raw[kCItems];
+#pragma unroll
+                for (int u = 0; u < kCItems; ++u) {
+                    const int q = tid + u * kThreads, i = q >> 5, c = q & 31;
+                    raw[u] = make_uint2(0u, 0u);
+                    if (i < T)
+                        raw[u] = __ldg(reinterpret_cast<const uint2 *>(p.C + (((size_t)b * T + i) * G + g) * kDstate + c * 4));
+                }
+#pragma unroll
+                for (int u = 0; u < kCItems; ++u) {
+                    const int q = tid + u * kThreads, i = q >> 5, c = q & 31;
+                    if (q < T_pad * 32) {
+                        float4 v;
+                        unpack4(raw[u], v.x, v.y, v.z, v.w);
+                        *reinterpret_cast<float4 *>(cs + (c >> 3) * T_pad * 128 + i * 128 + (((c & 7) ^ (i & 7)) << 4)) = v;
+                    }
+                }
+            }
+            if (new_b && !p.bs_mh)
                 for (uint32_t o = tid * 16u; o < (uint32_t)hpt * p.mh_head; o += kThreads * 16u)
                     *reinterpret_cast<float4 *>(mh + o) = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (tid == 0) {
-                    misc[M_LEN] = p.do_commit ? __ldg(&p.path_len[b]) : 0;
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (tid + u * kThreads < hpt * T) coef(k & 1, 0)[tid + u * kThreads] = bf2f(dtv[u]);
+            if (tid == 0) {
+                misc[M_DTK] = (int)k + 1;
+                if (new_b) {
+                    misc[M_LEN] = plen;
                     misc[M_STATE] = p.do_commit;
+                    if (!p.parent) misc[M_OK] = okv;
                 }
             }
+            ptx::cp_async_wait_all();
             __syncthreads();
             if (new_b) {
-                // Phase 2: the accepted path -- position q must hold the depth-q ancestor
-                // of the last node -- and the pair offsets (prefix sum of ancestor counts).
+                if (p.parent) {
+                    // Phase 2a: the tree itself -- node 0 the only root, every other
+                    // parent an earlier node -- then each node's ancestor-or-self row
+                    // and depth by walking its root path.  An invalid tree is reported
+                    // by the tree builder launched with this kernel; here its tiles
+                    // flow through the pipeline with empty masks and are not stored.
+                    int bad = 0;
+                    for (int i = tid; i < T; i += kThreads) {
+                        const int v = par[i];
+                        bad |= (i == 0) ? (v != -1) : (v < 0 || v >= i);
+                    }
+                    bad = __syncthreads_or(bad);
+                    for (int i = tid; i < T; i += kThreads) {
+                        for (int w = 0; w < W; ++w) ancs[i * W + w] = 0u;
+                        int d = -1;
+                        if (!bad)
+                            for (int j = i; j >= 0; j = par[j]) {
+                                ancs[i * W + (j >> 5)] |= 1u << (j & 31);
+                                ++d;
+                            }
+                        dep[i] = bad ? 0 : d;
+                    }
+                    if (tid == 0) misc[M_OK] = !bad;
+                    __syncthreads();
+                }
+                // Phase 2b: the accepted path -- position q must hold the depth-q
+                // ancestor of the last node -- and the pair offsets (prefix sum of
+                // ancestor counts).
                 const int len = misc[M_LEN];
-                if (p.do_commit) {
+                if (!misc[M_OK]) {
+                    if (tid == 0) misc[M_STATE] = 0;
+                } else if (p.do_commit) {
                     if (len < 0 || len > p.maxlen || len > T) {
                         if (tid == 0) {
                             misc[M_STATE] = 0;
                             latch_error(p.err, STREE_ERR_BAD_PATH, b, -1, len);
                         }
                     } else if (len > 0) {
-                        const int leaf = __ldg(&p.path[(size_t)b * p.maxlen + len - 1]);
+                        const int leaf = praw[len - 1];
                         const bool leaf_ok = leaf >= 0 && leaf < T;
                         for (int q = tid; q < len; q += kThreads) {
-                            const int j = __ldg(&p.path[(size_t)b * p.maxlen + q]);
+                            const int j = praw[q];
                             const bool good = leaf_ok && j >= 0 && j < T &&
-                                              ((ancs[leaf * W + (j >> 5)] >> (j & 31)) & 1u) &&
-                                              __ldg(&p.tree.depth[(size_t)b * T + j]) == q &&
-                                              (q != len - 1 || __ldg(&p.tree.depth[(size_t)b * T + leaf]) == len - 1);
+                                              ((ancs[leaf * W + (j >> 5)] >> (j & 31)) & 1u) && dep[j] == q &&
+                                              (q != len - 1 || dep[leaf] == len - 1);
                             if (!good) {
                                 misc[M_STATE] = 0;
                                 latch_error(p.err, STREE_ERR_BAD_PATH, b, q, j);
@@ -545,12 +652,29 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             __syncthreads();
             // Phase 3: path rows of B (fp32) for the commit, C_i . B_j of every ancestor pair.
-            if (misc[M_STATE]) {
+            if (misc[M_STATE] && p.tc_commit && misc[M_LEN] <= kPathRows) {
+                // B^T of the path rows, K-major fp32 (zeros past the path), for the commit MMA.
+                const int len = misc[M_LEN];
+                for (int it = tid; it < kDstate * 2; it += kThreads) {
+                    const int n = it & (kDstate - 1), kc = it >> 7;
+                    float v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = 4 * kc + e;
+                        const int j = q < len ? (int)pnode[q] : 0;
+                        const float bv = b_staged ? bf2f(Bs[j * kDstate + n]) : bf2f(Bseq[(size_t)j * brow + n]);
+                        v[e] = q < len ? bv : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(bts + k8_off(n, 4 * kc)) = make_float4(v[0], v[1], v[2], v[3]);
+                }
+            } else if (misc[M_STATE] && !p.tc_commit) {
                 const int nrows = min((int)misc[M_LEN], kPathRows);
                 for (int q = tid; q < nrows * 32; q += kThreads) {
+                    const int j = pnode[q >> 5];
+                    const uint2 raw = b_staged ? reinterpret_cast<const uint2 *>(Bs + j * kDstate)[q & 31]
+                                               : __ldg(reinterpret_cast<const uint2 *>(Bseq + (size_t)j * brow) + (q & 31));
                     float b0, b1, b2, b3;
-                    unpack4(__ldg(reinterpret_cast<const uint2 *>(Bseq + (size_t)pnode[q >> 5] * brow) + (q & 31)),
-                            b0, b1, b2, b3);
+                    unpack4(raw, b0, b1, b2, b3);
                     reinterpret_cast<float4 *>(Bp)[q] = make_float4(b0, b1, b2, b3);
                 }
             }
@@ -575,11 +699,17 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 for (int q0 = (tid >> 2); q0 < ((total + 7) & ~7); q0 += kThreads / 4) {
                     const int q = q0 < total ? q0 : total - 1;
                     const int i = pi[q], j = pj[q];
-                    float v = dot_cb_part(cs, T_pad, Bseq + (size_t)j * brow, i, part);
+                    float v = b_staged ? dot_cb_part<true>(cs, T_pad, Bs + j * kDstate, i, part)
+                                       : dot_cb_part<false>(cs, T_pad, Bseq + (size_t)j * brow, i, part);
                     v += __shfl_xor_sync(0xffffffffu, v, 1);
                     v += __shfl_xor_sync(0xffffffffu, v, 2);
                     if (part == 0 && q0 < total) pcb[q] = v;
                 }
+            }
+            if (p.bs_mh) {                                     // B rows read: clear the region for M_h
+                __syncthreads();
+                for (uint32_t o = tid * 16u; o < (uint32_t)hpt * p.mh_head; o += kThreads * 16u)
+                    *reinterpret_cast<float4 *>(mh + o) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
             ptx::fence_proxy_async_smem();
             __syncthreads();
@@ -588,6 +718,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         }
         const int len = misc[M_LEN];
         const bool commit = p.do_commit && misc[M_STATE];
+        const bool tcc = commit && p.tc_commit && len <= kPathRows;   // commit product on the tensor cores
         uint8_t *h0t = h0s + s * h0_stage_bytes;
         uint8_t *xt = xs + s * p.x_stage;
 
@@ -632,6 +763,17 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     ptx::mma_commit(bar(B_MHE));
                     STREE_TR(k, 3);
                 }
+                if (ok && tcc) {
+                    // Commit product D[row][n] = sum_q cf[row][q] B_q[n] (K = 8, tf32), once the
+                    // epilogue has written cf; the previous product was read before that.
+                    if (wait(bar(B_CFF), ncm & 1, 23)) {
+                        ptx::tc_fence_after();
+                        ptx::mma_tf32(tmem + (uint32_t)p.cm_col, ptx::desc_kmajor_none(ptx::smem_u32(cfs), 128, 256),
+                                      ptx::desc_kmajor_none(ptx::smem_u32(bts), 128, 256), ptx::idesc_tf32(RB, kDstate), 0);
+                        ptx::mma_commit(bar(B_CMF));
+                    }
+                }
+                if (tcc) ++ncm;
             }
         } else if (warp < kEpiWarp0) {
             // ------------------------------------------------------------ prep warps
@@ -646,10 +788,16 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             float *dts = coef(c, 0), *Ls = coef(c, 1), *eLs = coef(c, 2), *wts = coef(c, 3);
             float *alpha = coef(c, 4);
             if (ptid == 0) STREE_TR(k, 4);
-            if (ok) {
-                for (int q = ptid; q < hpt * T; q += kPrepThreads) {
-                    const int hh = q / T, i = q - hh * T;
-                    dts[q] = bf2f(p.dt[((size_t)b * T + i) * H + hfirst + hh]);
+            if (ok && misc[M_DTK] != (int)k + 1) {             // not already read by the switch
+                if (dnext_k == (int)k) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (ptid + u * kPrepThreads < hpt * T) dts[ptid + u * kPrepThreads] = bf2f(dnext[u]);
+                } else {
+                    for (int q = ptid; q < hpt * T; q += kPrepThreads) {
+                        const int hh = q / T, i = q - hh * T;
+                        dts[q] = bf2f(p.dt[((size_t)b * T + i) * H + hfirst + hh]);
+                    }
                 }
             }
             named_sync(kBarPrep, kPrepThreads);
@@ -684,7 +832,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 mbar_arrive(bar(B_COEFF + c));
                 if (ptid == 0) STREE_TR(k, 5);
                 // Masked decay matrix of every head of the tile (bf16, K-major swizzled):
-                // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i.
+                // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i,
+                // plus D_h on the diagonal, so that the tree MMA also yields the skip term.
                 if (ptid == 0 && k > 0) wait(bar(B_MHE), (k - 1) & 1, 32);
                 named_sync(kBarPrep, kPrepThreads);
                 ok = !misc[M_ABORT];
@@ -694,7 +843,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                         for (int q = ptid; q < hpt * total; q += kPrepThreads) {
                             const int hh = q / total, qq = q - hh * total;
                             const int i = pi[qq], j = pj[qq];
-                            const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * pcb[qq] * dts[hh * T + j];
+                            float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * pcb[qq] * dts[hh * T + j];
+                            if (i == j) m += Dsh[hfirst + hh];            // skip term D_h x_i
                             *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
                                 __float2bfloat16_rn(m);
                         }
@@ -703,8 +853,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                             const int hh = q / total, qq = q - hh * total;
                             const int i = pair_row(poff, T, qq);
                             const int j = nth_set_bit(ancs + i * W, W, qq - poff[i]);
-                            const float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) *
-                                            dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i) * dts[hh * T + j];
+                            float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) *
+                                      dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i) * dts[hh * T + j];
+                            if (i == j) m += Dsh[hfirst + hh];
                             *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
                                 __float2bfloat16_rn(m);
                         }
@@ -712,6 +863,17 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     ptx::fence_proxy_async_smem();
                     mbar_arrive(bar(B_MHF));
                     if (ptid == 0) STREE_TR(k, 6);
+                    // dt of the next tile when it belongs to the same (sequence, group)
+                    // (a switch reads its own); hpt * T <= 512 values.
+                    const int t1 = t + 1, b1 = t1 / p.tps, hf1 = (t1 % p.tps) * RB / P;
+                    if (t1 < end && b1 * G + hf1 / hpg == key) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int q = ptid + u * kPrepThreads, hh = q / T, i = q - hh * T;
+                            if (q < hpt * T) dnext[u] = p.dt[((size_t)b1 * T + i) * H + hf1 + hh];
+                        }
+                        dnext_k = (int)k + 1;
+                    }
                 }
             }
         } else {
@@ -730,17 +892,39 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             if (etid == 0) STREE_TR(k, 7);
             if (run) ptx::tc_fence_after();
             const float *eLs = coef(c, 2), *wts = coef(c, 3), *alpha = coef(c, 4);
-            if (run && commit) {
+            if (run && tcc) {
+                // Coefficients of the commit product: cf[row][q] = w_q x[pnode_q][row] for
+                // q < len, 0 past the path (K-major fp32, no swizzle).
+                for (int it = etid; it < RB * 2; it += kEpiThreads) {
+                    const int row = it % RB, kc = it / RB;
+                    const int hh = (r0 + row) / P - hfirst;
+                    const MnCol xc(row, xbs);
+                    float v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = 4 * kc + e;
+                        const int j = q < len ? (int)pnode[q] : 0;
+                        const float xv = bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
+                        v[e] = q < len ? wts[hh * T + q] * xv : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(cfs + k8_off(row, 4 * kc)) = make_float4(v[0], v[1], v[2], v[3]);
+                }
+                ptx::fence_proxy_async_smem();
+            } else if (run && commit) {
                 const int tpr = kEpiThreads / RB;                  // threads per row: 2 or 4
                 const int row = etid % RB, part = etid / RB;
                 const int hh = (r0 + row) / P - hfirst;
                 const MnCol xc(row, xbs);
                 const int cols = kDstate / tpr;
+                if (warp == 8 && lane == 0) STREE_TR(k, 20);
                 for (int c_lo = part * cols; c_lo < (part + 1) * cols; c_lo += 32)
-                    commit_rows<32>(h0t, xt, xc, Bp, Bseq, brow, pnode, wts + hh * T, alpha[hh], len, RB, row, c_lo);
+                    commit_rows<32>(h0t, xt, xc, Bp, p.tc_commit ? 0 : kPathRows, Bseq, brow, pnode, wts + hh * T,
+                                    alpha[hh], len, RB, row, c_lo);
+                if (warp == 8 && lane == 0) STREE_TR(k, 21);
             }
             if (warp == 8 && lane == 0) STREE_TR(k, 19);
             named_sync(kBarEpi, kEpiThreads);                  // x rows of the path are read
+            if (etid == 0 && run && tcc) mbar_arrive(bar(B_CFF));
             if (etid == 0) STREE_TR(k, 8);
             // A warp reads only its own quarter of the tensor-memory lanes: 32 * (warp % 4).
             // M = 128 puts tile row r in lane r; M = 64 puts rows 16q..16q+15 in
@@ -752,7 +936,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             const int row = RB == 128 ? quad * 32 + lane : quad * 16 + (lane & 15);
             if (run) {
                 const int hh = (r0 + row) / P - hfirst;           // same for the whole warp (P >= 32)
-                const float Dh = Dsh[hfirst + hh];
                 const float *eLh = eLs + hh * T;
                 const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * p.acc_cols);
                 const uint32_t ty = tl + (uint32_t)(T_pad * (1 + hh));
@@ -782,15 +965,12 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                         xa[u] = xbase + xc.at(i);
                         ea[u] = ebase + (uint32_t)i * 4u;
                     }
-                    uint16_t Xh[8];
                     float E[8];
-                    lds_u16x8(xa, Xh);
                     lds_f32x8(ea, E);
                     uint16_t Yh[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const float xv = __uint_as_float((uint32_t)Xh[u] << 16);
-                        const float yv = fmaf(E[u], __uint_as_float(R[u]), fmaf(Dh, xv, __uint_as_float(Y[u])));
+                        const float yv = fmaf(E[u], __uint_as_float(R[u]), __uint_as_float(Y[u]));
                         Yh[u] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
                     }
                     if (active && c0 + 8 <= T) {
@@ -812,6 +992,41 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 }
             }
             if (warp == 8 && lane == 0) STREE_TR(k, 16);
+            if (tcc) {
+                // h_new = alpha h0 + D, D read from tensor memory (same lane mapping as y).
+                if (etid == 0 && run) wait(bar(B_CMF), ncm & 1, 44);
+                named_sync(kBarEpi, kEpiThreads);
+                if (__all_sync(0xffffffffu, !misc[M_ABORT])) {
+                    ptx::tc_fence_after();
+                    const int hh = (r0 + row) / P - hfirst;
+                    const float2 a2 = make_float2(alpha[hh], alpha[hh]);
+                    const uint32_t td = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(p.cm_col + half * 64);
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        uint32_t d0[16], d1[16];
+                        ptx::tmem_ld16_nowait(td + (uint32_t)c0, d0);
+                        ptx::tmem_ld16_nowait(td + (uint32_t)(c0 + 16), d1);
+                        ptx::tmem_wait_ld();
+                        if (active) {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int n = half * 64 + c0 + 4 * u;
+                                const int kb = n >> 5, ch = (n & 31) >> 2;
+                                float4 *hp = reinterpret_cast<float4 *>(h0t + kb * RB * 128 + row * 128 +
+                                                                        ((ch ^ (row & 7)) << 4));
+                                const float4 h = *hp;
+                                const uint32_t *dv = u < 4 ? d0 + 4 * u : d1 + 4 * (u - 4);
+                                const float2 lo = ffma2(a2, make_float2(h.x, h.y),
+                                                        make_float2(__uint_as_float(dv[0]), __uint_as_float(dv[1])));
+                                const float2 hi = ffma2(a2, make_float2(h.z, h.w),
+                                                        make_float2(__uint_as_float(dv[2]), __uint_as_float(dv[3])));
+                                *hp = make_float4(lo.x, lo.y, hi.x, hi.y);
+                            }
+                        }
+                    }
+                }
+                ++ncm;
+            }
             ptx::tc_fence_before();
             __syncwarp();
             if (run && lane == 0) {
@@ -825,17 +1040,18 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             if (etid == 0) STREE_TR(k, 9);
             if (run && etid == 0) {
                 misc[M_SDESC + 2 * s] = t;                     // the producer issues the stores
-                misc[M_SDESC + 2 * s + 1] = commit ? 1 : 0;
+                misc[M_SDESC + 2 * s + 1] = (misc[M_OK] ? 1 : 0) | (commit ? 2 : 0);
                 mbar_arrive(bar(B_EPID + s));
             }
         }
-        ++k;
     }
 
     // ---------------------------------------------------------------- teardown
+    if (tid == 0) STREE_TR(31, 4);
     if (warp == kProducerWarp && lane == 0) {
         for (uint32_t q = stores_issued; q < k && !misc[M_ABORT]; ++q) store_tile(q);
         ptx::bulk_wait_all();
+        STREE_TR(31, 6);
         if (misc[M_ABORT]) {
             // Loads issued but never consumed may still land in this CTA's shared
             // memory: give them a bounded wait before the CTA exits.
@@ -848,7 +1064,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     if (warp == kMmaWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, p.tmem_cols);
+        if (lane == 0) STREE_TR(31, 5);
     }
+    // The grid completes no earlier than the launch it depends on (the tree
+    // builder), so later work on the stream sees both.
+    if (p.pre) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------------- host side
@@ -871,12 +1091,48 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+constexpr int kMaxDevices = 64;
+
+// Per-device facts looked up once: the SM count, and whether the kernel's
+// shared-memory limit has been raised on that device.
+struct DeviceInfo {
+    int sms = 0;
+    bool prepared = false;
+};
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
 int num_sms()
 {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < kMaxDevices) {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        if (g_dev[dev].sms > 0) return g_dev[dev].sms;
+    }
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    if (dev >= 0 && dev < kMaxDevices) {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        g_dev[dev].sms = n;
+    }
     return n;
+}
+
+// Raises the dynamic shared-memory limit of the kernel to the largest layout
+// (once per device; later launches need no attribute call).
+cudaError_t prepare_device()
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (g_dev[dev].prepared) return cudaSuccess;
+    e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    g_dev[dev].prepared = true;
+    return cudaSuccess;
 }
 
 uint32_t round_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -887,8 +1143,10 @@ struct TcPlan {
     int grid;
 };
 
-// Shared-memory layout for a tile height RB and S stages; false if it does not fit.
-bool layout(const ScanArgs &a, int RB, int S, TcParams &p, size_t &smem)
+// Shared-memory and tensor-memory layout for a tile height RB, S stages, (stage_b)
+// the B rows of a (sequence, group) kept in shared memory and (tcc) the commit
+// product on the tensor cores; false if it does not fit.
+bool layout(const ScanArgs &a, int RB, int S, bool stage_b, bool tcc, TcParams &p, size_t &smem)
 {
     const int T = a.T, T_pad = (T + 15) / 16 * 16, W = (T + 31) / 32;
     const int hpt = a.P >= RB ? 1 : RB / a.P;
@@ -907,12 +1165,37 @@ bool layout(const ScanArgs &a, int RB, int S, TcParams &p, size_t &smem)
     p.off_mh = round_up(off, 1024u);
     p.mh_head = (uint32_t)KA * T_pad * 128u;
     off = p.off_mh + (uint32_t)hpt * p.mh_head;
-    p.off_bp = round_up(off, 16u);     off = p.off_bp + (uint32_t)kPathRows * kDstate * 4u;
+    p.off_bp = 0;                      // fp32 path rows of B for the CUDA-core commit
+    if (!tcc) {
+        p.off_bp = round_up(off, 16u);
+        off = p.off_bp + (uint32_t)kPathRows * kDstate * 4u;
+    }
     p.off_anc = round_up(off, 16u);    off = p.off_anc + (uint32_t)T * W * 4u;
     p.off_poff = round_up(off, 16u);   off = p.off_poff + (uint32_t)(T + 1) * 4u;
     p.coef_slot = round_up((uint32_t)(4 * hpt * T + hpt) * 4u, 16u);
     p.off_coef = round_up(off, 16u);   off = p.off_coef + 2u * p.coef_slot;
     p.off_pnode = round_up(off, 16u);  off = p.off_pnode + (uint32_t)T * 2u;
+    p.off_praw = round_up(off, 16u);   off = p.off_praw + (uint32_t)T * 4u;
+    p.off_par = round_up(off, 16u);    off = p.off_par + (uint32_t)T * 4u;
+    p.off_dep = round_up(off, 16u);    off = p.off_dep + (uint32_t)T * 4u;
+    // B rows of a (sequence, group), bf16: a region of their own, else (when it
+    // is large enough) the masked-decay region, which is free during a switch.
+    p.off_bs = 0;
+    p.bs_mh = 0;
+    if (stage_b) {
+        p.off_bs = round_up(off, 16u);
+        off = p.off_bs + (uint32_t)T * kDstate * 2u;
+    } else if ((uint32_t)hpt * p.mh_head >= (uint32_t)T * kDstate * 2u) {
+        p.off_bs = p.off_mh;
+        p.bs_mh = 1;
+    }
+    p.off_cf = p.off_bt = 0;           // operands of the commit MMA (K = 8, fp32)
+    if (tcc) {
+        p.off_cf = round_up(off, 128u);
+        off = p.off_cf + (uint32_t)RB * 32u;
+        p.off_bt = round_up(off, 128u);
+        off = p.off_bt + (uint32_t)kDstate * 32u;
+    }
     p.off_bar = round_up(off, 16u);    off = p.off_bar + kNumBars * 8u;
     p.off_misc = round_up(off, 16u);   off = p.off_misc + kMiscWords * 4u;
     p.off_ad = round_up(off, 16u);     off = p.off_ad + 2u * a.H * 4u;
@@ -935,9 +1218,14 @@ bool layout(const ScanArgs &a, int RB, int S, TcParams &p, size_t &smem)
     p.NB = NB;
     p.S = S;
     p.hpt = hpt;
+    // Tensor memory: two accumulator sets (root term, tree term of each head), then
+    // the commit product (128 columns) when it runs on the tensor cores.
     p.acc_cols = (1 + hpt) * T_pad;
+    p.cm_col = 2 * p.acc_cols;
+    p.tc_commit = tcc ? 1 : 0;
+    const uint32_t need = (uint32_t)p.cm_col + (tcc ? (uint32_t)kDstate : 0u);
     uint32_t cols = 32;
-    while (cols < (uint32_t)(2 * p.acc_cols)) cols <<= 1;
+    while (cols < need) cols <<= 1;
     if (cols > 512) return false;
     p.tmem_cols = cols;
     return true;
@@ -966,11 +1254,18 @@ bool plan(const ScanArgs &a, TcPlan &pl)
     size_t best_smem = 0;
     for (const auto &c : cand) {
         const int RB = c[0], S = c[1];
+        if (!rb_valid(a, RB)) continue;
+        const int all_pairs = a.T * (a.T + 1) / 2;
         TcParams p{};
         size_t smem = 0;
-        if (!rb_valid(a, RB) || !layout(a, RB, S, p, smem)) continue;
-        const int all_pairs = a.T * (a.T + 1) / 2;
-        if (p.pair_cap < all_pairs && p.pair_cap < 4 * a.T) continue;   // typical trees must fit
+        bool fits = false;
+        // Preference: the commit product on the tensor cores, then B rows in a
+        // shared-memory region of their own.
+        for (int tcc = 1; tcc >= 0 && !fits; --tcc)
+            for (int stage_b = 1; stage_b >= 0 && !fits; --stage_b)
+                fits = layout(a, RB, S, stage_b != 0, tcc != 0, p, smem) &&
+                       (p.pair_cap >= all_pairs || p.pair_cap >= 4 * a.T);
+        if (!fits) continue;                                      // typical trees must fit
         const long long ntiles = (long long)a.batch * (a.H * a.P / RB);
         if (ntiles > 0x7fffffff) continue;
         if (ntiles >= sms) {
@@ -1019,6 +1314,8 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     p.path_len = a.path_len;
     p.maxlen = a.maxlen;
     p.do_commit = a.path != nullptr && a.h_new != nullptr;
+    p.parent = a.parent;
+    p.pre = a.parent != nullptr;
     p.tree = a.tree;
     p.err = a.err;
 
@@ -1056,20 +1353,14 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+    cudaError_t e = prepare_device();
     if (e != cudaSuccess) return e;
-    cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    int per_sm = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_tc_kernel, kThreads, pl.smem) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    // Tensor memory: every resident CTA holds tmem_cols of the SM's 512 columns.
-    const int tmem_fit = 512 / (int)p.tmem_cols;
-    if (per_sm > tmem_fit) per_sm = tmem_fit;
-    long long grid = (long long)num_sms() * per_sm;
+    // 448 threads at 128 registers leave room for one CTA per SM.
+    long long grid = num_sms();
     if (grid > p.ntiles) grid = p.ntiles;
-    // Programmatic dependent launch: the prologue (barriers, tensor memory, A/D)
-    // overlaps the preceding kernel, normally the tree builder.
+    // Programmatic dependent launch.  After the tree builder (parent given) the
+    // kernel needs nothing it writes and overlaps it entirely; otherwise the
+    // prologue (barriers, tensor memory) overlaps the tail of the preceding kernel.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);

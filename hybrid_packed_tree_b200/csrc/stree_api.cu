@@ -222,8 +222,10 @@ stree_status stree_tree_scan(stree_ctx *c, const void *x, const void *dt, const 
     if (st != STREE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((parent || batch == 0) && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
+    ScanArgs rec = a;
+    a.parent = parent;                      // the builder was launched right before
     if ((st = run_scan(c, a, s)) != STREE_OK) return st;
-    c->last = a;
+    c->last = rec;
     c->has_scan = true;
     return STREE_OK;
 }
@@ -264,6 +266,7 @@ stree_status stree_tree_scan_commit(stree_ctx *c, const void *x, const void *dt,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((parent || batch == 0) && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
     ScanArgs rec = a;
+    a.parent = parent;                      // the builder was launched right before
     a.path = path;
     a.path_len = path_len;
     a.maxlen = maxlen;

@@ -43,6 +43,10 @@ struct ScanArgs {
     int maxlen;
     float *h_new;
     TreeView tree;
+    // Set only when the tree builder was launched on the same stream right before
+    // the scan: the tensor-core kernel then builds the masks itself from parent[]
+    // and may read every input before that launch has finished.
+    const int32_t *parent;
     float *cb;                         // scratch [batch, G, T, T]: C_i . B_j on ancestor pairs
     int32_t *err;
 };

@@ -106,6 +106,20 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Asynchronous 4- and 8-byte global -> shared copies (they hold no registers
+// while in flight); cp_async_wait_all waits for all of this thread's copies.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(__cvta_generic_to_global(src)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(__cvta_generic_to_global(src)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -181,6 +195,17 @@ __device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, uint32_t (&r)[8]
                  : "r"(taddr));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns, no wait (pair with tmem_wait_ld).
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major operand in the canonical 128-byte
@@ -192,6 +217,17 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr)
            | ((uint64_t)(1024 >> 4) << 32)          // stride byte offset: 8 rows x 128 B
            | ((uint64_t)1 << 46)                    // descriptor version (sm_100)
            | ((uint64_t)2 << 61);                   // 128-byte swizzle
+}
+
+// Shared-memory matrix descriptor: K-major operand without swizzle: 8-row x
+// 16-byte core matrices of 128 contiguous bytes, `lbo` bytes between the core
+// matrices of adjacent K chunks, `sbo` bytes between adjacent 8-row groups.
+__device__ __forceinline__ uint64_t desc_kmajor_none(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4)
+           | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16)
+           | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32)
+           | ((uint64_t)1 << 46);                   // descriptor version; layout 0 = no swizzle
 }
 
 // Shared-memory matrix descriptor: MN-major operand in the canonical 128-byte

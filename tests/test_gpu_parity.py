@@ -251,6 +251,39 @@ def test_invalid_tree_latches_error_and_skips(st, bad):
     assert torch.isfinite(y[0]).all() and not torch.all(y[0] == 7.0)
 
 
+@pytest.mark.parametrize("rebuild", [True, False], ids=["parent", "ctx_tree"])
+@pytest.mark.parametrize("bad", [[-1, 0, 0, 0, 1, 1, 2, 2, 3, 3, 4, 5, 6, 7, 15],
+                                 [0, 0, 0, 0, 1, 1, 2, 2, 3, 3, 4, 5, 6, 7, 8],
+                                 [-1, 0, 0, 0, 1, 1, 2, 2, 3, 3, 4, 5, 6, 13, 8]])
+def test_tc_invalid_tree_skips_only_that_sequence(st, rebuild, bad):
+    """Tensor-core kernel (bf16, dstate 128) with an invalid middle sequence: its masks
+    built in-kernel from parent[] (parent passed) or read from the context's tree
+    (built by an earlier call).  The builder reports the tree; the kernel writes
+    neither y nor h_new of that sequence and the others stay exact."""
+    par = list(wl.M2_PARENT_15)
+    w = wl.custom_workload([par, par, par], nheads=4, headdim=64, dstate=128, dtype="bf16", seed=5, h0_std=0.1)
+    w.parent[1] = bad
+    ctx = _ctx(st, "tc")
+    d, tr = upload_layer(w), upload_tree(w)
+    y = torch.full_like(d["x"], 7.0)
+    h_new = torch.full_like(d["h0"], 7.0)
+    if not rebuild:
+        st.stree_build_tree(ctx, tr["parent"])
+    st.stree_tree_scan_commit(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"],
+                              tr["parent"] if rebuild else None, tr["path"], tr["path_len"], y, h_new)
+    status, info = st.stree_sync_check(ctx, raise_on_error=False)
+    assert status == 3 and info[1] == 1
+    assert torch.all(y[1] == 7.0) and torch.all(h_new[1] == 7.0)
+    f = w.f64(0)
+    keep = [0, 2]
+    sel = {k: (f[k][keep] if k in ("x", "dt", "B", "C", "h0") else f[k]) for k in f}
+    yr = oracle_tree_scan(sel["x"], sel["dt"], sel["A"], sel["B"], sel["C"], sel["D"], sel["h0"], w.parent[keep])
+    hr = oracle_commit(sel["x"], sel["dt"], sel["A"], sel["B"], sel["h0"], w.parent[keep], w.path[keep],
+                       w.path_len[keep])[0]
+    assert_close(f64(y[keep]), yr, "bf16", "y of the valid sequences")
+    assert_close(f64(h_new[keep]), hr, "bf16", "h_new of the valid sequences")
+
+
 @pytest.mark.parametrize("path,plen", [([1, 3, -1, -1], 2), ([0, 2, 3, -1], 3), ([0, 1, 3, 3], 5),
                                        ([0, 1, 3, 9], 4), ([0, 0, -1, -1], 2), ([0, 1, 3, -1], -1)])
 def test_invalid_path_latches_error(st, path, plen):
