@@ -49,7 +49,10 @@ constexpr int kMaxTcNodes = 128;           // T_pad <= 128 (TMEM columns, smem)
 constexpr int kPathRows = 8;               // accepted-path rows of B staged in smem (fp32)
 constexpr size_t kSmemLimit = 232448;      // 227 KB opt-in dynamic shared memory
 
-constexpr int kProducerWarp = 0, kMmaWarp = 1, kPrepWarp0 = 2, kPrepWarps = 4, kEpiWarp0 = 6, kEpiWarps = 8;
+// Sixteen warps at 128 registers fill the register file: producer, MMA issuer,
+// six prep warps, eight epilogue warps (two per tensor-memory lane quarter).
+constexpr int kProducerWarp = 0, kMmaWarp = 1, kPrepWarp0 = 2, kPrepWarps = 6;
+constexpr int kEpiWarp0 = kPrepWarp0 + kPrepWarps, kEpiWarps = 8;
 constexpr int kMaxStages = 3;
 constexpr int kMaxSmemHeads = 1024;        // A and D are staged in shared memory
 constexpr int kWarps = kEpiWarp0 + kEpiWarps;
@@ -61,11 +64,10 @@ enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_OK, M_DTK,
             kMiscWords = M_WSUM + kWarps };
 // mbarriers: TMA stage full / epilogue done with a stage (ring of S), tensor-memory
 // accumulator full / empty (ring of 2), masked-decay matrix full / empty,
-// per-tile coefficients full / empty (ring of 2), and for the tensor-core commit
-// its coefficient operand ready / its product done.
+// per-tile coefficients full / empty (ring of 2), and the tensor-core commit's
+// coefficient operand written.
 enum Bars { B_FULL = 0, B_EPID = kMaxStages, B_ACCF = 2 * kMaxStages, B_ACCE = B_ACCF + 2, B_MHF = B_ACCE + 2,
-            B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, B_CFF = B_COEFE + 2, B_CMF = B_CFF + 1,
-            kNumBars = B_CMF + 1 };
+            B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, B_CFF = B_COEFE + 2, kNumBars = B_CFF + 1 };
 
 struct TcParams {
     const __nv_bfloat16 *__restrict__ dt;
@@ -140,19 +142,22 @@ __device__ __forceinline__ float dot_cb(const uint8_t *cs, int T_pad, const __nv
 
 // C_i . B_j over the quarter `part` (32 of the 128 state columns); four lanes of
 // a warp combine their parts with shuffles.  B_j is read from shared memory
-// (kStaged) or from global memory.
+// (kStaged) or from global memory.  The eight pairs of a warp walk their 4-column
+// chunks in rotated order (`rot`): B rows lie 256 bytes apart, so the same chunk
+// of different rows would fall into the same shared-memory banks.
 template <bool kStaged>
-__device__ __forceinline__ float dot_cb_part(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i, int part)
+__device__ __forceinline__ float dot_cb_part(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i, int part,
+                                             int rot)
 {
     float acc = 0.f;
     const uint8_t *crow = cs + part * T_pad * 128 + i * 128;     // K-atom `part` holds columns 32*part..
     const uint2 *brow = reinterpret_cast<const uint2 *>(Bj) + part * 8;
     uint2 raw[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) raw[c] = kStaged ? brow[c] : __ldg(brow + c);
+    for (int c = 0; c < 8; ++c) raw[c] = kStaged ? brow[(c + rot) & 7] : __ldg(brow + ((c + rot) & 7));
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const float4 cv = *reinterpret_cast<const float4 *>(crow + ((c ^ (i & 7)) << 4));
+        const float4 cv = *reinterpret_cast<const float4 *>(crow + ((((c + rot) & 7) ^ (i & 7)) << 4));
         float b0, b1, b2, b3;
         unpack4(raw[c], b0, b1, b2, b3);
         acc = fmaf(cv.x, b0, acc);
@@ -445,8 +450,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         }
         ptx::mbar_init(bar(B_MHF), kPrepThreads);
         ptx::mbar_init(bar(B_MHE), 1);
-        ptx::mbar_init(bar(B_CFF), 1);
-        ptx::mbar_init(bar(B_CMF), 1);
+        ptx::mbar_init(bar(B_CFF), kPrepThreads);
         ptx::fence_mbar_init();
         for (int q = 0; q < kMiscWords; ++q) misc[q] = 0;
         for (uint32_t q = 0; q < npre; ++q) produce(q, start + (int)q);
@@ -502,6 +506,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             __syncthreads();                                   // every earlier tile is consumed
             if (tid == 0) STREE_TR(k, 12);
             const bool new_b = (b != cur_b);
+            [[maybe_unused]] const uint32_t swrow = cur_key < 0 ? 30u : 29u;   // trace row of this switch
             // Phase 1: every global read of this (sequence, group) in flight at once:
             // asynchronous copies for the B rows, parent, path, A and D (or the
             // context's tree), plain loads for dt and C (C is widened to fp32).
@@ -573,7 +578,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             ptx::cp_async_wait_all();
             __syncthreads();
+            if (tid == 0) STREE_TR(swrow, 0);
             if (new_b) {
+                bool okb;
                 if (p.parent) {
                     // Phase 2a: the tree itself -- node 0 the only root, every other
                     // parent an earlier node -- then each node's ancestor-or-self row
@@ -585,25 +592,27 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                         const int v = par[i];
                         bad |= (i == 0) ? (v != -1) : (v < 0 || v >= i);
                     }
-                    bad = __syncthreads_or(bad);
+                    okb = !__syncthreads_or(bad);
                     for (int i = tid; i < T; i += kThreads) {
                         for (int w = 0; w < W; ++w) ancs[i * W + w] = 0u;
                         int d = -1;
-                        if (!bad)
+                        if (okb)
                             for (int j = i; j >= 0; j = par[j]) {
                                 ancs[i * W + (j >> 5)] |= 1u << (j & 31);
                                 ++d;
                             }
-                        dep[i] = bad ? 0 : d;
+                        dep[i] = okb ? d : 0;
                     }
-                    if (tid == 0) misc[M_OK] = !bad;
+                    if (tid == 0) misc[M_OK] = okb;
                     __syncthreads();
+                } else {
+                    okb = misc[M_OK] != 0;
                 }
                 // Phase 2b: the accepted path -- position q must hold the depth-q
                 // ancestor of the last node -- and the pair offsets (prefix sum of
                 // ancestor counts).
                 const int len = misc[M_LEN];
-                if (!misc[M_OK]) {
+                if (!okb) {
                     if (tid == 0) misc[M_STATE] = 0;
                 } else if (p.do_commit) {
                     if (len < 0 || len > p.maxlen || len > T) {
@@ -651,6 +660,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 cur_b = b;
             }
             __syncthreads();
+            if (tid == 0) STREE_TR(swrow, 1);
             // Phase 3: path rows of B (fp32) for the commit, C_i . B_j of every ancestor pair.
             if (misc[M_STATE] && p.tc_commit && misc[M_LEN] <= kPathRows) {
                 // B^T of the path rows, K-major fp32 (zeros past the path), for the commit MMA.
@@ -680,6 +690,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             if (misc[M_INSMEM]) {
                 const int total = misc[M_TOTAL];
+                if (tid == 0) STREE_TR(swrow, 2);
                 // Node i's pairs: its ancestors in increasing order.
                 for (int i = tid; i < T; i += kThreads) {
                     int q = poff[i];
@@ -694,18 +705,21 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                 }
                 __syncthreads();
+                if (tid == 0) STREE_TR(swrow, 3);
                 // Four lanes per pair, a quarter of the state columns each.
                 const int part = lane & 3;
                 for (int q0 = (tid >> 2); q0 < ((total + 7) & ~7); q0 += kThreads / 4) {
                     const int q = q0 < total ? q0 : total - 1;
                     const int i = pi[q], j = pj[q];
-                    float v = b_staged ? dot_cb_part<true>(cs, T_pad, Bs + j * kDstate, i, part)
-                                       : dot_cb_part<false>(cs, T_pad, Bseq + (size_t)j * brow, i, part);
+                    const int rot = (lane >> 2) & 7;
+                    float v = b_staged ? dot_cb_part<true>(cs, T_pad, Bs + j * kDstate, i, part, rot)
+                                       : dot_cb_part<false>(cs, T_pad, Bseq + (size_t)j * brow, i, part, rot);
                     v += __shfl_xor_sync(0xffffffffu, v, 1);
                     v += __shfl_xor_sync(0xffffffffu, v, 2);
                     if (part == 0 && q0 < total) pcb[q] = v;
                 }
             }
+            if (tid == 0) STREE_TR(swrow, 4);
             if (p.bs_mh) {                                     // B rows read: clear the region for M_h
                 __syncthreads();
                 for (uint32_t o = tid * 16u; o < (uint32_t)hpt * p.mh_head; o += kThreads * 16u)
@@ -759,19 +773,25 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                                          ptx::desc_kmajor_sw128(mb + (ks >> 2) * T_pad * 128 + (ks & 3) * 32),
                                          idesc_tree, ks != 0);
                     }
-                    ptx::mma_commit(bar(B_ACCF + a));
-                    ptx::mma_commit(bar(B_MHE));
-                    STREE_TR(k, 3);
-                }
-                if (ok && tcc) {
-                    // Commit product D[row][n] = sum_q cf[row][q] B_q[n] (K = 8, tf32), once the
-                    // epilogue has written cf; the previous product was read before that.
-                    if (wait(bar(B_CFF), ncm & 1, 23)) {
-                        ptx::tc_fence_after();
-                        ptx::mma_tf32(tmem + (uint32_t)p.cm_col, ptx::desc_kmajor_none(ptx::smem_u32(cfs), 128, 256),
-                                      ptx::desc_kmajor_none(ptx::smem_u32(bts), 128, 256), ptx::idesc_tf32(RB, kDstate), 0);
-                        ptx::mma_commit(bar(B_CMF));
+                    if (tcc) {
+                        // Commit product D[row][n] = sum_q cf[row][q] B_q[n] (K = 8, tf32) once the
+                        // prep warps have written cf.  The epilogue read the previous product
+                        // before this tile's accumulator became free.
+                        ok = wait(bar(B_CFF), ncm & 1, 23);
+                        if (ok) {
+                            ptx::tc_fence_after();
+                            ptx::mma_tf32(tmem + (uint32_t)p.cm_col,
+                                          ptx::desc_kmajor_none(ptx::smem_u32(cfs), 128, 256),
+                                          ptx::desc_kmajor_none(ptx::smem_u32(bts), 128, 256),
+                                          ptx::idesc_tf32(RB, kDstate), 0);
+                        }
                     }
+                    if (ok) {
+                        // Tile accumulators (and the commit product) full; M_h and cf free.
+                        ptx::mma_commit(bar(B_ACCF + a));
+                        ptx::mma_commit(bar(B_MHE));
+                    }
+                    STREE_TR(k, 3);
                 }
                 if (tcc) ++ncm;
             }
@@ -874,6 +894,32 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                         }
                         dnext_k = (int)k + 1;
                     }
+                    if (tcc) {
+                        // Coefficients of the commit product, once the tile's x has landed:
+                        // cf[row][q] = w_q x[pnode_q][row] for q < len, 0 past the path
+                        // (K-major fp32, no swizzle).  The previous product was read by its
+                        // MMA before this tile's M_h region was released.
+                        if (ptid == 0) wait(bar(B_FULL + s), sph, 33);
+                        named_sync(kBarPrep, kPrepThreads);
+                        if (!misc[M_ABORT]) {
+                            for (int it = ptid; it < RB * 2; it += kPrepThreads) {
+                                const int row = it % RB, kc = it / RB;
+                                const int hh = (r0 + row) / P - hfirst;
+                                const MnCol xc(row, xbs);
+                                float v[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int q = 4 * kc + e;
+                                    const int j = q < len ? (int)pnode[q] : 0;
+                                    const float xv = bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
+                                    v[e] = q < len ? wts[hh * T + q] * xv : 0.f;
+                                }
+                                *reinterpret_cast<float4 *>(cfs + k8_off(row, 4 * kc)) = make_float4(v[0], v[1], v[2], v[3]);
+                            }
+                            ptx::fence_proxy_async_smem();
+                            mbar_arrive(bar(B_CFF));
+                        }
+                    }
                 }
             }
         } else {
@@ -892,25 +938,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             if (etid == 0) STREE_TR(k, 7);
             if (run) ptx::tc_fence_after();
             const float *eLs = coef(c, 2), *wts = coef(c, 3), *alpha = coef(c, 4);
-            if (run && tcc) {
-                // Coefficients of the commit product: cf[row][q] = w_q x[pnode_q][row] for
-                // q < len, 0 past the path (K-major fp32, no swizzle).
-                for (int it = etid; it < RB * 2; it += kEpiThreads) {
-                    const int row = it % RB, kc = it / RB;
-                    const int hh = (r0 + row) / P - hfirst;
-                    const MnCol xc(row, xbs);
-                    float v[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int q = 4 * kc + e;
-                        const int j = q < len ? (int)pnode[q] : 0;
-                        const float xv = bf2f(*reinterpret_cast<const __nv_bfloat16 *>(xt + xc.at(j)));
-                        v[e] = q < len ? wts[hh * T + q] * xv : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(cfs + k8_off(row, 4 * kc)) = make_float4(v[0], v[1], v[2], v[3]);
-                }
-                ptx::fence_proxy_async_smem();
-            } else if (run && commit) {
+            if (run && commit && !tcc) {
                 const int tpr = kEpiThreads / RB;                  // threads per row: 2 or 4
                 const int row = etid % RB, part = etid / RB;
                 const int hh = (r0 + row) / P - hfirst;
@@ -924,7 +952,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             if (warp == 8 && lane == 0) STREE_TR(k, 19);
             named_sync(kBarEpi, kEpiThreads);                  // x rows of the path are read
-            if (etid == 0 && run && tcc) mbar_arrive(bar(B_CFF));
             if (etid == 0) STREE_TR(k, 8);
             // A warp reads only its own quarter of the tensor-memory lanes: 32 * (warp % 4).
             // M = 128 puts tile row r in lane r; M = 64 puts rows 16q..16q+15 in
@@ -992,11 +1019,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 }
             }
             if (warp == 8 && lane == 0) STREE_TR(k, 16);
-            if (tcc) {
+            if (tcc && run) {
                 // h_new = alpha h0 + D, D read from tensor memory (same lane mapping as y).
-                if (etid == 0 && run) wait(bar(B_CMF), ncm & 1, 44);
-                named_sync(kBarEpi, kEpiThreads);
-                if (__all_sync(0xffffffffu, !misc[M_ABORT])) {
+                {
                     ptx::tc_fence_after();
                     const int hh = (r0 + row) / P - hfirst;
                     const float2 a2 = make_float2(alpha[hh], alpha[hh]);
@@ -1025,7 +1050,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                         }
                     }
                 }
-                ++ncm;
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -1355,7 +1379,7 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     }
     cudaError_t e = prepare_device();
     if (e != cudaSuccess) return e;
-    // 448 threads at 128 registers leave room for one CTA per SM.
+    // 512 threads at 128 registers leave room for one CTA per SM.
     long long grid = num_sms();
     if (grid > p.ntiles) grid = p.ntiles;
     // Programmatic dependent launch.  After the tree builder (parent given) the
