@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=None, help="override the workload's layer count (profiling)")
     ap.add_argument("--also", default="serve64",
                     help="comma-separated extra workloads summarised in the same line ('none' to skip)")
+    ap.add_argument("--no-unrolled", action="store_true",
+                    help="skip the unrolled-tree baseline comparison (one layer per workload)")
     return ap.parse_args()
 
 
@@ -189,6 +191,69 @@ def dev_tensor(torch, a, io, device):
     if io == "bf16":
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def run_unrolled(name, local_rank, steps=5):
+    """The unrolled-tree baseline on one layer of a workload: every root-to-leaf path
+    scanned as its own sequence with its own state (stree_unrolled_scan), timed as a
+    CUDA graph of `steps` launches after an L2 flush."""
+    import torch
+
+    from hybrid_packed_tree_b200 import stree
+    from hybrid_packed_tree_b200 import workloads as wl
+
+    device = torch.device("cuda", local_rank)
+    w = wl.make_workload(name, layers=1)
+    paths, plen = wl.unroll_paths(w.parent)
+    L, io = w.layers[0], w.dtype
+    d = {k: dev_tensor(torch, getattr(L, k), io, device) for k in ("x", "dt", "B", "C")}
+    d.update({k: dev_tensor(torch, getattr(L, k), "f32", device) for k in ("A", "D", "h0")})
+    pt, lt = torch.from_numpy(paths).to(device), torch.from_numpy(plen).to(device)
+    b, n_paths, depth = paths.shape
+    y = torch.empty((b, n_paths, depth, w.nheads, w.headdim), dtype=d["x"].dtype, device=device)
+    h = torch.empty((b, n_paths, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=device)
+    err = torch.zeros(4, dtype=torch.int32, device=device)
+
+    def call():
+        stree.stree_unrolled_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], pt, lt, y, h,
+                                  err_out=err, stream=torch.cuda.current_stream(device))
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(steps):
+            call()
+    g.replay()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(int(3 * l2) // 4 + 1, dtype=torch.float32, device=device)
+    flush.zero_()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    g.replay()
+    t1.record()
+    torch.cuda.synchronize(device)
+    if int(err[0]) != 0:
+        raise RuntimeError(f"device error in the unrolled baseline: {err.tolist()}")
+    ms = t0.elapsed_time(t1) / steps
+    del g
+    state = w.nheads * w.headdim * w.dstate * 4
+    real = int((plen > 0).sum())
+    return {"workload": name, "layers": 1, "ms_per_launch": ms, "paths": real, "path_positions": int(plen.sum()),
+            "tree_nodes": w.batch * w.n_nodes, "path_state_bytes": real * state,
+            "nodes_per_s": w.batch * w.n_nodes / (ms / 1e3)}
+
+
+def unrolled_summary(o, u):
+    """Unrolled baseline beside the packed scan (per layer: the packed step time
+    divided by the layers)."""
+    packed_ms = o["ms_per_step"] / o["config"]["layers"]
+    u = dict(u)
+    u["packed_ms_per_layer"] = packed_ms
+    u["unrolled_over_packed_time"] = u["ms_per_launch"] / packed_ms
+    return u
 
 
 def run_ours(args, rank, world, local_rank):
@@ -496,6 +561,10 @@ def main():
                 "roofline": {k: r2[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic",
                                                 "bytes_per_launch", "kernel_ms_mean")},
             }
+            if not args.no_unrolled and rank == 0:
+                out["other_workloads"][name]["unrolled_baseline"] = unrolled_summary(o2, run_unrolled(name, local_rank))
+    if rank == 0 and not args.no_unrolled:
+        out["unrolled_baseline"] = unrolled_summary(out, run_unrolled(args.config, local_rank))
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_seconds)
     if rank == 0:

@@ -39,7 +39,7 @@ EXPORTS = (
     "stree_ctx_create", "stree_ctx_destroy", "stree_ctx_set_kernel", "stree_ctx_launch_count",
     "stree_build_tree",
     "stree_tree_scan", "stree_commit", "stree_tree_scan_commit", "stree_tree_scan_commit_noalloc",
-    "stree_resolve_path",
+    "stree_resolve_path", "stree_unrolled_scan",
     "stree_sync_check", "stree_status_string", "stree_version",
 )
 
@@ -54,6 +54,7 @@ _lib.stree_commit.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
 _lib.stree_tree_scan_commit.argtypes = [_vp] * 9 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp]
 _lib.stree_tree_scan_commit_noalloc.argtypes = [_vp] * 8 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp, _vp]
 _lib.stree_resolve_path.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
+_lib.stree_unrolled_scan.argtypes = [_vp] * 9 + [_i] * 9 + [_vp, _vp, _vp, _vp]
 _lib.stree_sync_check.argtypes = [_vp, _vp, _ip]
 _lib.stree_status_string.argtypes = [_i]
 _lib.stree_status_string.restype = ctypes.c_char_p
@@ -221,6 +222,24 @@ def stree_tree_scan_commit_noalloc(x, dt, A, B, C, D, h0, parent, path, path_len
                                              _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
     _check(st, "stree_tree_scan_commit_noalloc")
     return y, h_new
+
+
+def stree_unrolled_scan(x, dt, A, B, C, D, h0, paths, path_len, y_paths, h_paths, err_out=None, stream=None):
+    """(y_paths, h_paths) <- every path scanned as its own sequence (the unrolled-tree baseline).
+
+    paths [b, n_paths, max_depth] int32, path_len [b, n_paths] int32,
+    y_paths [b, n_paths, max_depth, H, P] in x's dtype, h_paths [b, n_paths, H, P, N] fp32.
+    """
+    ins, yp = _scan_ptrs(x, dt, A, B, C, D, h0, y_paths)
+    batch, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    st = _lib.stree_unrolled_scan(*ins[:7], _ptr(paths, "paths", (torch.int32,)),
+                                  _ptr(path_len, "path_len", (torch.int32,)), T, batch, paths.shape[1],
+                                  paths.shape[2], H, P, N, G, _io_dtype(x), yp,
+                                  _ptr(h_paths, "h_paths", (torch.float32,)),
+                                  _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
+    _check(st, "stree_unrolled_scan")
+    return y_paths, h_paths
 
 
 def stree_resolve_path(ctx: Ctx, path, path_len, leaf_out, stream=None):

@@ -141,6 +141,24 @@ def leaves(parent_row) -> np.ndarray:
     return np.nonzero(~has_child)[0]
 
 
+def unroll_paths(parent: np.ndarray):
+    """Every root-to-leaf path of each sequence's tree (the unrolled form of the
+    tree), leaves in increasing order, padded to the largest leaf count with
+    empty paths.  Returns paths [b, n_paths, max_depth] int32 (-1 past each
+    path's end) and path_len [b, n_paths] int32."""
+    parent = np.asarray(parent)
+    per_seq = [[root_path_nodes(row, int(l)) for l in leaves(row)] for row in parent]
+    n_paths = max(len(ps) for ps in per_seq)
+    max_depth = max(len(p) for ps in per_seq for p in ps)
+    paths = np.full((len(per_seq), n_paths, max_depth), -1, np.int32)
+    path_len = np.zeros((len(per_seq), n_paths), np.int32)
+    for b, ps in enumerate(per_seq):
+        for k, nodes in enumerate(ps):
+            paths[b, k, :len(nodes)] = nodes
+            path_len[b, k] = len(nodes)
+    return paths, path_len
+
+
 # --------------------------------------------------------------------------- workloads
 
 

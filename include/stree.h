@@ -173,6 +173,35 @@ stree_status stree_tree_scan_commit_noalloc(const void *x, const void *dt, const
                                             int32_t *err_out, void *stream);
 
 /*
+ * Unrolled-tree baseline (STree summary, "Problem" and "Key results": the
+ * alternative the packed tree is compared with).  Every given path -- normally
+ * each root-to-leaf path of the draft tree -- is scanned as its own sequence with
+ * the plain recurrence, s <- exp(dt_k A_h) s + dt_k x_k (outer) B_k and
+ * y_k = s . C_k + D_h x_k from h0, and keeps its own final state.  Nodes shared by
+ * several paths are recomputed once per path.  No context is used.
+ *
+ *   x, dt, A, B, C, D, h0: as for stree_tree_scan (n_nodes nodes per sequence)
+ *   paths    [batch, n_paths, max_depth] int32 node ids, first node first
+ *   path_len [batch, n_paths] int32, 0 <= len <= max_depth (entries past len ignored)
+ *   y_paths  [batch, n_paths, max_depth, nheads, headdim] in x's dtype: y of the
+ *            node at each position (positions >= len untouched)
+ *   h_paths  [batch, n_paths, nheads, headdim, dstate] fp32: each path's final state
+ *            (h0 itself for an empty path)
+ *   err_out  device int32[4] error word of this call (cleared by the call), or NULL
+ *
+ * A path with a length out of range or a node id outside [0, n_nodes) latches
+ * STREE_ERR_BAD_PATH and leaves that path's outputs untouched.  Shapes: headdim a
+ * multiple of 8 and dstate a multiple of 16, both up to 256; n_nodes and
+ * max_depth up to 256 (else STREE_ERR_UNSUPPORTED).  The caller owns every
+ * buffer; the call allocates nothing and runs on `stream`.
+ */
+stree_status stree_unrolled_scan(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                                 const float *D, const float *h0, const int32_t *paths, const int32_t *path_len,
+                                 int n_nodes, int batch, int n_paths, int max_depth, int nheads, int headdim,
+                                 int dstate, int ngroups, stree_dtype dtype, void *y_paths, float *h_paths,
+                                 int32_t *err_out, void *stream);
+
+/*
  * Resolve accepted paths against the context's current tree: leaf_out[b] (device
  * int32 [batch]) receives the last node of a valid path, -1 for an empty path and
  * -2 for an invalid one (which also latches STREE_ERR_BAD_PATH).

@@ -377,3 +377,23 @@ def test_pins_catch_planted_mistakes(mutant, tmp_path):
           np.asarray(m["h0"]).reshape(1, 1, 2, 3), np.asarray([m["parent"]], np.int32))
     caught.append(not np.allclose(run(*mc).reshape(2, 2), m["y"], atol=1e-12))
     assert any(caught), f"no pin caught the planted mistake: {mutant}"
+
+
+def test_unroll_paths_lists_every_root_to_leaf_chain():
+    """Host-side unrolling used by the unrolled baseline: one path per leaf, each a
+    chain from the root (parent[path[k]] == path[k-1]) ending at that leaf."""
+    rng = np.random.default_rng(11)
+    parents = np.stack([wl.random_tree(rng, 40, max_depth=6) for _ in range(3)])
+    paths, plen = wl.unroll_paths(parents)
+    for b in range(3):
+        lv = set(int(l) for l in wl.leaves(parents[b]))
+        got = set()
+        for k in range(paths.shape[1]):
+            n = int(plen[b, k])
+            if n == 0:
+                continue
+            nodes = paths[b, k, :n]
+            assert nodes[0] == 0 and parents[b][nodes[0]] == -1
+            assert all(parents[b][nodes[q]] == nodes[q - 1] for q in range(1, n))
+            got.add(int(nodes[-1]))
+        assert got == lv and sum(plen[b] > 0) == len(lv)
