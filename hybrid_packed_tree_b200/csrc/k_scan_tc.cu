@@ -64,10 +64,11 @@ enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_OK, M_DTK,
             kMiscWords = M_WSUM + kWarps };
 // mbarriers: TMA stage full / epilogue done with a stage (ring of S), tensor-memory
 // accumulator full / empty (ring of 2), masked-decay matrix full / empty,
-// per-tile coefficients full / empty (ring of 2), and the tensor-core commit's
-// coefficient operand written.
+// per-tile coefficients full / empty (ring of 2), and for the tensor-core commit
+// its coefficient operand written and its (single) product read.
 enum Bars { B_FULL = 0, B_EPID = kMaxStages, B_ACCF = 2 * kMaxStages, B_ACCE = B_ACCF + 2, B_MHF = B_ACCE + 2,
-            B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, B_CFF = B_COEFE + 2, kNumBars = B_CFF + 1 };
+            B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, B_CFF = B_COEFE + 2, B_CME = B_CFF + 1,
+            kNumBars = B_CME + 1 };
 
 struct TcParams {
     const __nv_bfloat16 *__restrict__ dt;
@@ -451,6 +452,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         ptx::mbar_init(bar(B_MHF), kPrepThreads);
         ptx::mbar_init(bar(B_MHE), 1);
         ptx::mbar_init(bar(B_CFF), kPrepThreads);
+        ptx::mbar_init(bar(B_CME), kEpiWarps);
         ptx::fence_mbar_init();
         for (int q = 0; q < kMiscWords; ++q) misc[q] = 0;
         for (uint32_t q = 0; q < npre; ++q) produce(q, start + (int)q);
@@ -775,9 +777,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     if (tcc) {
                         // Commit product D[row][n] = sum_q cf[row][q] B_q[n] (K = 8, tf32) once the
-                        // prep warps have written cf.  The epilogue read the previous product
-                        // before this tile's accumulator became free.
-                        ok = wait(bar(B_CFF), ncm & 1, 23);
+                        // prep warps have written cf and the epilogue has read the previous
+                        // product (D has one buffer).
+                        ok = (ncm == 0 || wait(bar(B_CME), (ncm - 1) & 1, 24)) && wait(bar(B_CFF), ncm & 1, 23);
                         if (ok) {
                             ptx::tc_fence_after();
                             ptx::mma_tf32(tmem + (uint32_t)p.cm_col,
@@ -1050,6 +1052,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                         }
                     }
                 }
+                // This warp's reads of the commit product are done: the next one may be issued.
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_CME));
             }
             ptx::tc_fence_before();
             __syncwarp();
