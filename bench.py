@@ -54,6 +54,10 @@ def parse():
                     help="comma-separated extra workloads summarised in the same line ('none' to skip)")
     ap.add_argument("--no-unrolled", action="store_true",
                     help="skip the unrolled-tree baseline comparison (one layer per workload)")
+    ap.add_argument("--no-accept", action="store_true",
+                    help="skip the greedy tree-verification timing (argmax over the logits + walk)")
+    ap.add_argument("--vocab", type=int, default=50280,
+                    help="vocabulary of the synthetic logits for the verification timing (Mamba2-2.7B's padded vocab)")
     return ap.parse_args()
 
 
@@ -244,6 +248,65 @@ def run_unrolled(name, local_rank, steps=5):
     return {"workload": name, "layers": 1, "ms_per_launch": ms, "paths": real, "path_positions": int(plen.sum()),
             "tree_nodes": w.batch * w.n_nodes, "path_state_bytes": real * state,
             "nodes_per_s": w.batch * w.n_nodes / (ms / 1e3)}
+
+
+def run_accept(name, vocab, local_rank, steps=20):
+    """Greedy tree verification (stree_accept_greedy) on synthetic bf16 logits
+    [b, T, vocab] of a workload's trees, timed as a CUDA graph of `steps` calls after
+    an L2 flush.  Its bytes are the logits (argmax) plus the small tree inputs."""
+    import torch
+
+    from hybrid_packed_tree_b200 import stree
+    from hybrid_packed_tree_b200 import workloads as wl
+
+    device = torch.device("cuda", local_rank)
+    w = wl.make_workload(name, layers=1)
+    b, T = w.batch, w.n_nodes
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1234)
+    # Distinct logits per call (up to `steps` copies, enough that no call finds its
+    # logits in L2 after the flush).
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nsets = max(1, min(steps, -(-3 * l2 // (b * T * vocab * 2))))
+    logit_sets = [torch.randn((b, T, vocab), generator=gen, device=device).to(torch.bfloat16) for _ in range(nsets)]
+    tokens = torch.randint(0, vocab, (b, T), generator=gen, device=device, dtype=torch.int32)
+    parent = torch.from_numpy(w.parent).to(device)
+    pred = torch.empty((b, T), dtype=torch.int32, device=device)
+    path = torch.empty((b, T), dtype=torch.int32, device=device)
+    plen = torch.empty((b,), dtype=torch.int32, device=device)
+    bonus = torch.empty((b,), dtype=torch.int32, device=device)
+    err = torch.zeros(4, dtype=torch.int32, device=device)
+
+    def call(i):
+        stree.stree_accept_greedy(logit_sets[i % nsets], tokens, parent, pred, path, plen, bonus, err_out=err,
+                                  stream=torch.cuda.current_stream(device))
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            call(i)
+    g.replay()
+    flush = torch.empty(int(3 * l2) // 4 + 1, dtype=torch.float32, device=device)
+    flush.zero_()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    g.replay()
+    t1.record()
+    torch.cuda.synchronize(device)
+    if int(err[0]) != 0:
+        raise RuntimeError(f"device error in the verification step: {err.tolist()}")
+    ms = t0.elapsed_time(t1) / steps
+    del g
+    nbytes = b * T * vocab * 2 + b * T * 4 * 3 + b * T * 4 + b * 8
+    hbm_gbs, peak_kind = peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": name, "vocab": vocab, "logits_dtype": "bf16", "ms_per_call": ms, "bytes_per_call": nbytes,
+            "achieved_gbs": gbs, "frac": gbs / hbm_gbs, "peak_source": f"{peak_kind} hbm_gbs",
+            "timing": f"{steps} calls in one CUDA graph after an L2 flush, {nsets} distinct logits buffers"}
 
 
 def unrolled_summary(o, u):
@@ -563,8 +626,12 @@ def main():
             }
             if not args.no_unrolled and rank == 0:
                 out["other_workloads"][name]["unrolled_baseline"] = unrolled_summary(o2, run_unrolled(name, local_rank))
+            if not args.no_accept and rank == 0:
+                out["other_workloads"][name]["accept_greedy"] = run_accept(name, args.vocab, local_rank)
     if rank == 0 and not args.no_unrolled:
         out["unrolled_baseline"] = unrolled_summary(out, run_unrolled(args.config, local_rank))
+    if rank == 0 and not args.no_accept:
+        out["accept_greedy"] = run_accept(args.config, args.vocab, local_rank)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_seconds)
     if rank == 0:

@@ -39,7 +39,7 @@ EXPORTS = (
     "stree_ctx_create", "stree_ctx_destroy", "stree_ctx_set_kernel", "stree_ctx_launch_count",
     "stree_build_tree",
     "stree_tree_scan", "stree_commit", "stree_tree_scan_commit", "stree_tree_scan_commit_noalloc",
-    "stree_resolve_path", "stree_unrolled_scan",
+    "stree_resolve_path", "stree_unrolled_scan", "stree_accept_greedy",
     "stree_sync_check", "stree_status_string", "stree_version",
 )
 
@@ -55,6 +55,7 @@ _lib.stree_tree_scan_commit.argtypes = [_vp] * 9 + [_i] * 7 + [_vp, _vp, _i, _vp
 _lib.stree_tree_scan_commit_noalloc.argtypes = [_vp] * 8 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp, _vp]
 _lib.stree_resolve_path.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
 _lib.stree_unrolled_scan.argtypes = [_vp] * 9 + [_i] * 9 + [_vp, _vp, _vp, _vp]
+_lib.stree_accept_greedy.argtypes = [_vp, _i, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.stree_sync_check.argtypes = [_vp, _vp, _ip]
 _lib.stree_status_string.argtypes = [_i]
 _lib.stree_status_string.restype = ctypes.c_char_p
@@ -240,6 +241,22 @@ def stree_unrolled_scan(x, dt, A, B, C, D, h0, paths, path_len, y_paths, h_paths
                                   _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
     _check(st, "stree_unrolled_scan")
     return y_paths, h_paths
+
+
+def stree_accept_greedy(logits, draft_tokens, parent, pred, accepted_path, path_len, bonus_token, err_out=None,
+                        stream=None):
+    """Greedy tree verification: (pred, accepted_path, path_len, bonus_token) from the
+    target's logits [b, T, V] (fp32 or bf16) and the draft tokens [b, T]."""
+    batch, T, V = logits.shape
+    st = _lib.stree_accept_greedy(_ptr(logits, "logits", (torch.float32, torch.bfloat16)), _io_dtype(logits), V,
+                                  _ptr(draft_tokens, "draft_tokens", (torch.int32,)),
+                                  _ptr(parent, "parent", (torch.int32,)), T, batch, accepted_path.shape[1],
+                                  _ptr(pred, "pred", (torch.int32,)), _ptr(accepted_path, "accepted_path", (torch.int32,)),
+                                  _ptr(path_len, "path_len", (torch.int32,)),
+                                  _ptr(bonus_token, "bonus_token", (torch.int32,)),
+                                  _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
+    _check(st, "stree_accept_greedy")
+    return pred, accepted_path, path_len, bonus_token
 
 
 def stree_resolve_path(ctx: Ctx, path, path_len, leaf_out, stream=None):

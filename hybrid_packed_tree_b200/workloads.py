@@ -159,6 +159,35 @@ def unroll_paths(parent: np.ndarray):
     return paths, path_len
 
 
+def acceptance_inputs(parent: np.ndarray, vocab: int, seed: int = 7, dtype: str = "bf16"):
+    """Synthetic target logits and draft tokens for tree verification: tokens
+    distinct among each node's children, logits ~ N(0,1) with, along one random
+    root-to-leaf path per sequence, the next node's token raised above the row's
+    maximum (so that a greedy verifier follows that path) and one raised token after
+    the leaf.  Returns (logits [b,T,V] fp32 or bf16 bits, tokens [b,T] int32,
+    planted paths as lists)."""
+    parent = np.asarray(parent)
+    rng = np.random.default_rng(seed)
+    b, T = parent.shape
+    tokens = np.zeros((b, T), np.int32)
+    logits = rng.normal(size=(b, T, vocab)).astype(np.float32)
+    planted = []
+    for s_ in range(b):
+        for u in range(T):
+            kids = np.nonzero(parent[s_] == u)[0]
+            if len(kids):
+                tokens[s_, kids] = rng.choice(vocab, size=len(kids), replace=False)
+        leaf = int(rng.choice(leaves(parent[s_])))
+        nodes = root_path_nodes(parent[s_], leaf)
+        for u, v in zip(nodes[:-1], nodes[1:]):
+            logits[s_, u, tokens[s_, v]] = logits[s_, u].max() + 1.0
+        logits[s_, leaf, int(rng.integers(vocab))] = logits[s_, leaf].max() + 1.0
+        planted.append(nodes)
+    if dtype == "bf16":
+        logits = bf16_bits(logits)
+    return logits, tokens, planted
+
+
 # --------------------------------------------------------------------------- workloads
 
 

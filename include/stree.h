@@ -202,6 +202,33 @@ stree_status stree_unrolled_scan(const void *x, const void *dt, const float *A, 
                                  int32_t *err_out, void *stream);
 
 /*
+ * Greedy (temperature 0) verification of the draft tree (STree summary, "Key
+ * results" at temperature 0; "Builds on": SpecInfer, speculative sampling).  The
+ * target's prediction after node i is pred[i] = argmax_v logits[i][v] (ties: the
+ * smaller token id).  From the root, a child is accepted when its draft token
+ * equals the prediction after its parent (equal sibling tokens: the smaller node
+ * index), and the walk continues from it, for at most maxlen nodes.  The result
+ * is exactly the accepted_path / path_len that stree_commit takes.
+ *
+ *   logits        [batch, n_nodes, vocab] fp32 or bf16 (logit_dtype), finite
+ *   draft_tokens  [batch, n_nodes] int32: the token of each node (root's unused)
+ *   parent        [batch, n_nodes] int32: the packed tree (as for the scan)
+ *   pred_out      [batch, n_nodes] int32: receives pred
+ *   accepted_path [batch, maxlen] int32: receives the root-first accepted nodes, -1 after
+ *   path_len      [batch] int32: receives the number of accepted nodes (>= 1)
+ *   bonus_token   [batch] int32: receives pred of the last accepted node
+ *   err_out       device int32[4] error word of this call (cleared by the call), or NULL
+ *
+ * An invalid tree latches STREE_ERR_BAD_TREE for that sequence and gives it
+ * path_len 0, bonus -1 and a path of -1.  n_nodes up to 256.  The caller owns every
+ * buffer; the call allocates nothing and runs on `stream`.
+ */
+stree_status stree_accept_greedy(const void *logits, stree_dtype logit_dtype, int vocab,
+                                 const int32_t *draft_tokens, const int32_t *parent, int n_nodes, int batch,
+                                 int maxlen, int32_t *pred_out, int32_t *accepted_path, int32_t *path_len,
+                                 int32_t *bonus_token, int32_t *err_out, void *stream);
+
+/*
  * Resolve accepted paths against the context's current tree: leaf_out[b] (device
  * int32 [batch]) receives the last node of a valid path, -1 for an empty path and
  * -2 for an invalid one (which also latches STREE_ERR_BAD_PATH).

@@ -397,3 +397,52 @@ def test_unroll_paths_lists_every_root_to_leaf_chain():
             assert all(parents[b][nodes[q]] == nodes[q - 1] for q in range(1, n))
             got.add(int(nodes[-1]))
         assert got == lv and sum(plen[b] > 0) == len(lv)
+
+
+# ------------------------------------------------------------------ greedy acceptance
+
+
+def test_accept_greedy_golden_cases():
+    """Hand-worked cases (tests/golden/accept_greedy.json): ties, equal sibling
+    tokens, no match, a full chain and the maxlen cut."""
+    from oracle import oracle_accept_greedy
+    with open(os.path.join(os.path.dirname(__file__), "golden", "accept_greedy.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        lg = np.asarray(c["logits"], np.float64)[None]
+        pred, path, plen, bonus = oracle_accept_greedy(lg, np.asarray(c["tokens"])[None],
+                                                       np.asarray(c["parent"])[None], c["maxlen"])
+        n = c["path_len"]
+        assert int(plen[0]) == n, c["name"]
+        assert path[0, :n].tolist() == c["path"], c["name"]
+        assert (path[0, n:] == -1).all(), c["name"]
+        assert int(bonus[0]) == c["bonus"], c["name"]
+
+
+def test_accept_greedy_follows_a_planted_path():
+    """Random trees with distinct sibling tokens and logits whose maximum after
+    every node of a chosen root-to-leaf path is the next node's token: exactly
+    that path is accepted, and the bonus is the token planted after the leaf."""
+    from oracle import oracle_accept_greedy
+    rng = np.random.default_rng(21)
+    b, T, V = 5, 30, 97
+    parents = np.stack([wl.random_tree(rng, T, max_depth=6) for _ in range(b)])
+    tokens = np.zeros((b, T), np.int64)
+    logits = rng.normal(size=(b, T, V))
+    want_paths, want_bonus = [], []
+    for s in range(b):
+        for u in range(T):                        # distinct tokens among each node's children
+            kids = [c for c in range(T) if parents[s, c] == u]
+            tokens[s, kids] = rng.choice(V, size=len(kids), replace=False)
+        leaf = int(rng.choice(wl.leaves(parents[s])))
+        nodes = wl.root_path_nodes(parents[s], leaf)
+        for u, v in zip(nodes[:-1], nodes[1:]):
+            logits[s, u, tokens[s, v]] = logits[s, u].max() + 1.0
+        bonus_tok = int(rng.integers(V))
+        logits[s, leaf, bonus_tok] = logits[s, leaf].max() + 1.0
+        want_paths.append(nodes)
+        want_bonus.append(bonus_tok)
+    pred, path, plen, bonus = oracle_accept_greedy(logits, tokens, parents, T)
+    for s in range(b):
+        assert path[s, :plen[s]].tolist() == want_paths[s]
+        assert int(bonus[s]) == want_bonus[s]
