@@ -42,6 +42,13 @@
  * of 8 in [8, 256], nheads a multiple of ngroups.  Pointers to tensors must be
  * 16-byte aligned.  batch = 0 is a no-op that returns STREE_OK.
  *
+ * Precision: all accumulation is fp32.  The CUDA-core kernel (STREE_KERNEL_SIMT,
+ * and every fp32 input) computes in fp32 throughout.  The tensor-core kernel
+ * (bf16 inputs, dstate 128, n_nodes <= 128, headdim a multiple of 32) rounds h0 to
+ * tf32 in the root term, the masked decay matrix (D_h on its diagonal included) to
+ * bf16, and the commit coefficients dt-weighted x to tf32; each rounding is below
+ * the bf16 rounding of y itself.
+ *
  * Ownership and threading: the caller owns every tensor.  A context (stree_ctx)
  * owns the library's device workspace (tree masks, depths, per-sequence flags,
  * the error word, a C.B scratch for the tree term).  Workspace is allocated by
@@ -75,7 +82,7 @@ typedef enum {
     STREE_ERR_BAD_PATH = 4,     /* device-detected: accepted path is not a root->node chain */
     STREE_ERR_MISALIGNED = 5,   /* a tensor pointer is not 16-byte aligned */
     STREE_ERR_CUDA = 6,         /* a CUDA runtime call failed (launch, allocation) */
-    STREE_ERR_TIMEOUT = 7,      /* a bounded device wait gave up (reserved) */
+    STREE_ERR_TIMEOUT = 7,      /* a bounded wait inside the tensor-core kernel gave up (about 1 s) */
     STREE_ERR_NO_TREE = 8       /* scan with parent = NULL before any tree was built, or
                                    commit before any scan, or a size mismatch with them */
 } stree_status;
