@@ -9,8 +9,8 @@ load or call it, and the two share no code.
 * ``packed`` -- a second fp64 formulation (numpy) of the same outputs through the
                accumulated transition ``A_tree = L . log A``; used only to
                cross-check the walk.
-* ``accept`` -- greedy (temperature 0) verification of the draft tree: the
-               accepted path and bonus token from the target's logits.
+* ``accept`` -- verification of the draft tree: greedy (temperature 0) and by
+               multi-step speculative sampling; the accepted path and bonus token.
 """
 from .walk import (  # noqa: F401
     build_oracle,
@@ -19,4 +19,4 @@ from .walk import (  # noqa: F401
     oracle_max_threads,
     oracle_tree_scan,
 )
-from .accept import oracle_accept_greedy  # noqa: F401,E402
+from .accept import oracle_accept_greedy, oracle_accept_sampling  # noqa: F401,E402

@@ -446,3 +446,62 @@ def test_accept_greedy_follows_a_planted_path():
     for s in range(b):
         assert path[s, :plen[s]].tolist() == want_paths[s]
         assert int(bonus[s]) == want_bonus[s]
+
+
+# ------------------------------------------------------------------ sampling acceptance
+
+
+def test_accept_sampling_golden_cases():
+    """Hand-worked cases (tests/golden/accept_sampling.json): acceptance with
+    probability p/q, the residual after a rejection, a second sibling accepted
+    against the residual, bonus tokens by inverse CDF."""
+    from oracle import oracle_accept_sampling
+    with open(os.path.join(os.path.dirname(__file__), "golden", "accept_sampling.json")) as f:
+        doc = json.load(f)
+    for c in doc["cases"]:
+        path, plen, bonus = oracle_accept_sampling(
+            np.asarray(c["target_logits"])[None], np.asarray(c["draft_logits"])[None], np.asarray(c["tokens"])[None],
+            np.asarray(c["parent"])[None], doc["temperature"], np.asarray(c["u_accept"])[None],
+            np.asarray([c["u_bonus"]]), c["maxlen"])
+        n = c["path_len"]
+        assert int(plen[0]) == n and path[0, :n].tolist() == c["path"], c["name"]
+        assert int(bonus[0]) == c["bonus"], c["name"]
+
+
+def test_accept_sampling_at_vanishing_temperature_is_greedy():
+    """As the temperature goes to 0 both distributions become one-hot on their
+    argmax: a child is accepted exactly when its token is the target's argmax,
+    and the bonus is that argmax -- the greedy rule."""
+    from oracle import oracle_accept_greedy, oracle_accept_sampling
+    w = wl.make_workload("serve64", batch=6, layers=1)
+    logits, tokens, _ = wl.acceptance_inputs(w.parent, 64, seed=13, dtype="f32")
+    rng = np.random.default_rng(14)
+    draft = rng.normal(size=logits.shape)
+    ua = rng.uniform(size=tokens.shape)
+    ub = rng.uniform(size=w.batch) * 0.999
+    g_pred, g_path, g_len, g_bonus = oracle_accept_greedy(logits, tokens, w.parent, w.n_nodes)
+    s_path, s_len, s_bonus = oracle_accept_sampling(logits, draft, tokens, w.parent, 1e-4, ua, ub, w.n_nodes)
+    assert np.array_equal(g_path, s_path) and np.array_equal(g_len, s_len) and np.array_equal(g_bonus, s_bonus)
+
+
+def test_accept_sampling_first_token_follows_the_target_distribution():
+    """Losslessness: with the root's children drawn independently from the draft
+    distribution q, the first token emitted (the accepted child's token, else the
+    bonus) is distributed as the target's p, whatever q is (Monte Carlo, 5 sigma)."""
+    from oracle import oracle_accept_sampling
+    rng = np.random.default_rng(15)
+    V, k, n = 5, 3, 30000
+    p = np.array([0.35, 0.05, 0.25, 0.15, 0.20])
+    q = np.array([0.10, 0.40, 0.10, 0.30, 0.10])
+    tl = np.zeros((n, k + 1, V))
+    tl[:, 0] = np.log(p)
+    dl = np.zeros((n, k + 1, V))
+    dl[:, 0] = np.log(q)
+    tokens = np.zeros((n, k + 1), np.int64)
+    tokens[:, 1:] = rng.choice(V, size=(n, k), p=q)
+    parent = np.tile(np.array([-1] + [0] * k), (n, 1))
+    path, plen, bonus = oracle_accept_sampling(tl, dl, tokens, parent, 1.0, rng.uniform(size=(n, k + 1)),
+                                               rng.uniform(size=n), k + 1)
+    first = np.where(plen >= 2, tokens[np.arange(n), np.maximum(path[:, 1], 0)], bonus)
+    freq = np.bincount(first, minlength=V) / n
+    assert np.all(np.abs(freq - p) < 5 * np.sqrt(p * (1 - p) / n)), (freq, p)
