@@ -191,6 +191,14 @@ def weak_scaling_value(units_per_rank_step, steps, ms, world):
 # ----------------------------------------------------------------------------- our arm
 
 
+def workload_config(name, batch=None, layers=None):
+    """The workload keys of the JSON line's `config` (the same for both arms)."""
+    from hybrid_packed_tree_b200 import workloads as wl
+    _, b0, l0, H, P, N, G, T, io, _ = wl.SPECS[name]
+    return {"workload": name, "batch": batch or b0, "layers": layers or l0, "n_nodes": T, "nheads": H,
+            "headdim": P, "dstate": N, "ngroups": G, "io_dtype": io, "state_dtype": "f32"}
+
+
 def dev_tensor(torch, a, io, device):
     if io == "bf16":
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
@@ -445,8 +453,7 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if io == "bf16" else "f32", "data": "synthetic (seeded; shapes and distributions of the workload)",
         "config": {
-            "workload": args.config, "batch": w.batch, "layers": nl, "n_nodes": w.n_nodes, "nheads": w.nheads,
-            "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "io_dtype": io, "state_dtype": "f32",
+            **workload_config(args.config, args.batch, args.layers),
             "kernel": args.kernel, "parallelism": f"replicas x{world}",
             "l2": (f"rotates {nsets} buffer copies ({nsets * step_bytes / 2**20:.0f} MiB > 3x L2)"
                    if nsets > 1 else "step bytes exceed L2 (no reuse between steps)")
@@ -580,7 +587,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": K,
         "warmup": Wm, "ms_per_step": el * 1e3 / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": args.config, "sample": desc},
+        "config": {**workload_config(args.config, args.batch, args.layers), "sample": desc},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
