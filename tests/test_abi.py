@@ -114,3 +114,38 @@ def test_noalloc_rejects_oversized_scratch_on_the_host(lib_path):
     fake = 0x10000                                    # aligned, never dereferenced
     args = [fake] * 8 + [256, 1 << 16, 8, 64, 128, 1, 1] + [fake, fake, 256, fake, fake, None, None]
     assert fn(*args) == 2
+
+
+def test_unrolled_and_accept_host_checks(lib_path):
+    """Shape, dtype, pointer and alignment checks of stree_unrolled_scan and
+    stree_accept_greedy happen on the host, before any device work."""
+    from hybrid_packed_tree_b200 import stree
+    un = stree._lib.stree_unrolled_scan
+    ok = 0x10000                                      # aligned, never dereferenced
+    # x, dt, A, B, C, D, h0, paths, path_len; T, batch, n_paths, max_depth, H, P, N, G, dtype; y, h, err, stream
+    base = [ok] * 9 + [15, 1, 6, 4, 80, 64, 128, 1, 1] + [ok, ok, None, None]
+
+    def call(fn, args, **over):
+        a = list(args)
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return fn(*a)
+
+    assert call(un, base, i9=0) == 2                  # n_nodes 0
+    assert call(un, base, i11=0) == 2                 # n_paths 0
+    assert call(un, base, i15=120) == 2               # dstate not a multiple of 16
+    assert call(un, base, i16=3) == 2                 # 80 heads over 3 groups
+    assert call(un, base, i17=7) == 2                 # unknown dtype
+    assert call(un, base, i18=ok + 4) == 5            # y misaligned
+    assert call(un, base, i0=None) == 1               # x missing
+    assert call(un, base, i0=ok + 8) == 5             # x misaligned
+    assert call(un, base, i10=0) == 0                 # batch 0: nothing to do
+    acc = stree._lib.stree_accept_greedy
+    # logits, dtype, V, tokens, parent, T, batch, maxlen, pred, path, len, bonus, err, stream
+    abase = [ok, 1, 50280, ok, ok, 15, 1, 15, ok, ok, ok, ok, None, None]
+    assert call(acc, abase, i5=257) == 2              # more than 256 nodes
+    assert call(acc, abase, i1=5) == 2                # unknown logits dtype
+    assert call(acc, abase, i7=0) == 2                # maxlen 0
+    assert call(acc, abase, i9=None) == 1             # no path buffer
+    assert call(acc, abase, i0=ok + 1) == 5           # bf16 logits on an odd address
+    assert call(acc, abase, i6=0) == 0                # batch 0: nothing to do
