@@ -2,9 +2,9 @@
 
 The algorithmic bytes are the denominator-free half of the roofline: every tensor
 of one fused launch moved once (h0 and h_new fp32, x and y in the input dtype, dt,
-B, C, A, D, the tree and the path).  They are checked against the figures of the
-scope table (m2_2p7b 5.56 MB, hyb8b 37.8 MB, serve64 422 MB per layer, wide256
-1.63 GB) and against a direct recount from the tensor shapes.
+B, C, A, D, the tree and the path).  They are checked against the workloads' byte
+counts worked out by hand (m2_2p7b 5.56 MB, hyb8b 37.8 MB, serve64 422 MB per
+layer, wide256 1.63 GB) and against a direct recount from the tensor shapes.
 """
 import os
 import sys
@@ -20,7 +20,7 @@ from hybrid_packed_tree_b200 import workloads as wl  # noqa: E402
 
 
 @pytest.mark.parametrize("name,mb", [("m2_2p7b", 5.56), ("hyb8b", 37.8), ("serve64", 422.0), ("wide256", 1630.0)])
-def test_algorithmic_bytes_match_the_scope_table(name, mb):
+def test_algorithmic_bytes_match_the_hand_counts(name, mb):
     w = wl.make_workload(name, layers=1)
     total = sum(bench.algorithmic_bytes(w).values())
     assert abs(total / 1e6 - mb) / mb < 0.01, (name, total)
