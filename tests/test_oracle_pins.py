@@ -505,3 +505,42 @@ def test_accept_sampling_first_token_follows_the_target_distribution():
     first = np.where(plen >= 2, tokens[np.arange(n), np.maximum(path[:, 1], 0)], bonus)
     freq = np.bincount(first, minlength=V) / n
     assert np.all(np.abs(freq - p) < 5 * np.sqrt(p * (1 - p) / n)), (freq, p)
+
+
+def test_accept_pins_catch_planted_mistakes():
+    """Copies of the verification oracles with one planted mistake each must fail
+    the pins above: last-index ties, the largest matching child, no maxlen cut, no
+    residual after a rejection, a bonus from the undisturbed target distribution."""
+    import oracle.accept as acc
+    src = open(acc.__file__).read()
+    mutants = {
+        "ties to the larger id": ("pred = np.argmax(logits, axis=-1).astype(np.int64)",
+                                  "pred = (logits.shape[-1] - 1 - np.argmax(logits[..., ::-1], axis=-1)).astype(np.int64)"),
+        "largest matching child": ("for c in range(T):                       # children in increasing index order",
+                                   "for c in reversed(range(T)):             # children in decreasing index order"),
+        "no maxlen cut": ("        while len(nodes) < maxlen:\n", "        while True:\n"),
+        "no residual": ("                    r = np.maximum(p - q, 0.0)\n                    if r.sum() > 0.0:\n                        p = r / r.sum()\n",
+                        "                    pass\n"),
+        "bonus from the target": ("        cdf = np.cumsum(p)\n", "        cdf = np.cumsum(_softmax(tl[s, cur] / temperature))\n"),
+    }
+    checks = [test_accept_greedy_golden_cases, test_accept_greedy_follows_a_planted_path,
+              test_accept_sampling_golden_cases, test_accept_sampling_at_vanishing_temperature_is_greedy,
+              test_accept_sampling_first_token_follows_the_target_distribution]
+    import oracle
+    for name, (old, new) in mutants.items():
+        assert src.count(old) == 1, name
+        ns = {"__name__": "mutant"}
+        exec(compile(src.replace(old, new), "mutant", "exec"), ns)
+        saved = (oracle.oracle_accept_greedy, oracle.oracle_accept_sampling)
+        oracle.oracle_accept_greedy, oracle.oracle_accept_sampling = ns["oracle_accept_greedy"], ns["oracle_accept_sampling"]
+        try:
+            caught = False
+            for chk in checks:
+                try:
+                    chk()
+                except (AssertionError, IndexError, ValueError):
+                    caught = True
+                    break
+            assert caught, f"mutant '{name}' passed every pin"
+        finally:
+            oracle.oracle_accept_greedy, oracle.oracle_accept_sampling = saved
