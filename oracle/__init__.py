@@ -11,6 +11,8 @@ load or call it, and the two share no code.
                cross-check the walk.
 * ``accept`` -- verification of the draft tree: greedy (temperature 0) and by
                multi-step speculative sampling; the accepted path and bonus token.
+* ``attention`` -- tree-masked attention of the hybrid model's Transformer layers
+               over the packed tree (context plus each node's root path).
 """
 from .walk import (  # noqa: F401
     build_oracle,
@@ -20,3 +22,4 @@ from .walk import (  # noqa: F401
     oracle_tree_scan,
 )
 from .accept import oracle_accept_greedy, oracle_accept_sampling  # noqa: F401,E402
+from .attention import oracle_tree_attention  # noqa: F401,E402
