@@ -34,6 +34,11 @@ if ROOT not in sys.path:
 METRIC = "tree-scan nodes/sec and achieved HBM GB/s (% of roofline), 1×B200"
 UNIT = "nodes/s"
 DEFAULT_CONFIG = "m2_2p7b"
+# Extra workloads that also get an end-to-end figure, and that also run the
+# unrolled baseline and the verification timing (the wide trees would need tens
+# of GB of per-path states unrolled).
+E2E_WORKLOADS = ("serve64",)
+SIDE_WORKLOADS = ("m2_2p7b", "hyb8b", "serve64")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -44,14 +49,16 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
-    ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tc", "small"], default="auto")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample budget")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--layers", type=int, default=None, help="override the workload's layer count (profiling)")
-    ap.add_argument("--also", default="serve64",
+    ap.add_argument("--also", default="hyb8b,serve64,wide256,wide256_chain",
                     help="comma-separated extra workloads summarised in the same line ('none' to skip)")
+    ap.add_argument("--no-separate", action="store_true",
+                    help="skip the stand-alone scan and commit timings")
     ap.add_argument("--no-unrolled", action="store_true",
                     help="skip the unrolled-tree baseline comparison (one layer per workload)")
     ap.add_argument("--no-accept", action="store_true",
@@ -99,22 +106,39 @@ def source_sha(fname):
 
 
 def profile_traffic(kernel_name, workload):
-    """Per-launch DRAM bytes (read + write) of the dominant kernel for this workload,
-    from the committed ncu summary, if it was taken on the current kernel source;
-    else None."""
-    summ = os.path.join(ROOT, "profiles", "traffic.md")
-    if not os.path.exists(summ):
+    """Per-launch DRAM bytes (read + write) of a kernel on this workload, from the
+    committed ncu figures (profiles/traffic.json), if they were taken on the current
+    kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
         return None
-    for line in open(summ):
-        if not line.startswith("traffic:"):
+    with open(path) as f:
+        entries = json.load(f).get("entries", [])
+    for e in entries:
+        if e.get("kernel") != kernel_name or e.get("workload") != workload:
             continue
-        kv = dict(t.split("=", 1) for t in line[len("traffic:"):].split())
-        if kv.get("kernel") != kernel_name or kv.get("workload") != workload:
-            continue
-        if source_sha(kv.get("file", "")) != kv.get("sha"):
+        if source_sha(e.get("file", "")) != e.get("sha"):
             return None
-        return float(kv["bytes_per_launch"])
+        return float(e["bytes_per_launch"])
     return None
+
+
+KERNEL_NAMES = {"small": "scan_small_kernel", "tc": "scan_tc_kernel", "simt": "scan_simt_kernel"}
+
+
+def commit_bytes(w):
+    """Bytes of one stand-alone commit launch (one layer): h0 read, h_new written,
+    the path, and x, dt and B at the accepted path's nodes."""
+    b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    e = 2 if w.dtype == "bf16" else 4
+    nodes = int(np.sum(w.path_len))
+    return 2 * b * H * P * N * 4 + b * w.maxlen * 4 + b * 4 + nodes * (H * P * e + H * e + G * N * e)
+
+
+def scan_bytes(w):
+    """Bytes of one stand-alone scan launch (one layer): every input once and y."""
+    a = algorithmic_bytes(w)
+    return sum(v for k, v in a.items() if k not in ("h_new", "path"))
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -436,18 +460,37 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     kern_ms = [e[0].elapsed_time(e[1]) for per in evs for e in per]
-    del g_steps, g_events, flush
+    del g_steps, g_events
+    kernel_used = stree.stree_ctx_last_kernel(ctx)
+    sep = None
+    if not args.no_separate:
+        sep = run_separate(torch, stree, w, ctx, sets, nsets, K, device, flush)
+    del flush
     st, info = stree.stree_sync_check(ctx, stream, raise_on_error=False)
     if st != 0:
         raise RuntimeError(f"device error during the benchmark: {info}")
 
     ms, kmean = max_over_ranks([ms, statistics.mean(kern_ms)], world, device)
+    if sep is not None:
+        sep["scan"]["ms_per_launch"], sep["commit"]["ms_per_launch"] = max_over_ranks(
+            [sep["scan"]["ms_per_launch"], sep["commit"]["ms_per_launch"]], world, device)
+        hbm_gbs0, _ = peaks()
+        for part in (sep["scan"], sep["commit"]):
+            part["achieved_gbs"] = part["bytes_per_launch"] / (part["ms_per_launch"] / 1e3) / 1e9
+            part["frac"] = part["achieved_gbs"] / hbm_gbs0
 
     nodes_step = w.batch * w.n_nodes * nl
     value = weak_scaling_value(nodes_step, K, ms, world)
     hbm_gbs, peak_kind = peaks()
-    achieved = launch_bytes / (kmean / 1e3) / 1e9
-    kernel_name = "scan_tc_kernel" if args.kernel != "simt" else "scan_simt_kernel"
+    kernel_name = KERNEL_NAMES.get(kernel_used, kernel_used)
+    step_gbs = step_bytes * K / (ms / 1e3) / 1e9
+    # The kernel's average launch duration: when the step graph holds nothing but
+    # one launch of it per layer, the timed region over the launch count; else the
+    # mean of the event pairs around every launch (those event nodes also end the
+    # overlap of consecutive launches, so they read a little high).
+    only_scan = int(launches) == K * nl
+    launch_ms = ms / (K * nl) if only_scan else kmean
+    achieved = launch_bytes / (launch_ms / 1e3) / 1e9
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -460,23 +503,72 @@ def run_ours(args, rank, world, local_rank):
                   + "; 3x-L2 buffer written before each timed replay",
             "timing": "CUDA graph of the K steps, replayed once (CUDA events around the replay)",
         },
-        "hbm": {"step_bytes": step_bytes, "gbs_step": step_bytes * K / (ms / 1e3) / 1e9},
+        "hbm": {"step_bytes": step_bytes, "gbs_step": step_gbs},
         "sequences_per_s": world * w.batch * K / (ms / 1e3),
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
             "frac": achieved / hbm_gbs, "traffic": profile_traffic(kernel_name, args.config),
             "peak_source": f"{peak_kind} hbm_gbs", "kernel": kernel_name,
-            "bytes_per_launch": launch_bytes, "kernel_ms_mean": kmean,
-            "kernel_ms_median": statistics.median(kern_ms),
+            "bytes_per_launch": launch_bytes, "kernel_ms_mean": launch_ms,
+            "launch_ms_from": "step graph / launches" if only_scan else "events around every launch",
+            "kernel_ms_events": kmean, "kernel_ms_events_median": statistics.median(kern_ms),
+            "achieved_events": launch_bytes / (kmean / 1e3) / 1e9,
+            "frac_events": launch_bytes / (kmean / 1e3) / 1e9 / hbm_gbs,
         },
         "clocks": clk,
         "gpu_launches": int(launches),
     }
+    if sep is not None:
+        out["separate"] = sep
 
     if not args.no_e2e:
         out["e2e"] = e2e(torch, stree, w, ctx, device, stream, args, world)
     stree.stree_ctx_destroy(ctx)
     return out
+
+
+def run_separate(torch, stree, w, ctx, sets, nsets, K, device, flush):
+    """The stand-alone scan (stree_tree_scan) and commit (stree_commit) of every layer,
+    each call bracketed by timing events inside one CUDA graph of K steps, replayed
+    after an L2 flush.  Returns per-launch means and the algorithmic bytes of each."""
+    nl = w.nlayers
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(K * nl)]
+
+    def step(i):
+        layers, tree = sets[i % nsets]
+        s = torch.cuda.current_stream(device)
+        for li, d in enumerate(layers):
+            e = ev[i * nl + li]
+            e[0].record(s)
+            stree.stree_tree_scan(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"],
+                                  tree["parent"] if li == 0 else None, d["y"], stream=s)
+            e[1].record(s)
+            e[2].record(s)
+            stree.stree_commit(ctx, tree["path"], tree["path_len"], d["h_new"], stream=s)
+            e[3].record(s)
+
+    step(0)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(K):
+            step(i)
+    g.replay()
+    flush.zero_()
+    torch.cuda.synchronize(device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    scan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    commit_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    kernel_used = stree.stree_ctx_last_kernel(ctx)
+    del g
+    return {
+        "scan": {"kernel": KERNEL_NAMES.get(kernel_used, kernel_used), "ms_per_launch": scan_ms,
+                 "bytes_per_launch": scan_bytes(w)},
+        "commit": {"kernel": "commit_kernel", "ms_per_launch": commit_ms, "bytes_per_launch": commit_bytes(w)},
+        "timing": f"{K} steps x {nl} layers of scan-then-commit in one CUDA graph after an L2 flush, "
+                  "timing events around every call",
+    }
 
 
 def e2e(torch, stree, w, ctx, device, stream, args, world):
@@ -622,18 +714,24 @@ def main():
         out["other_workloads"] = {}
         for name in extras:
             a2 = copy.copy(args)
-            a2.config, a2.no_e2e, a2.steps, a2.batch, a2.layers = name, True, None, None, None
+            a2.config, a2.steps, a2.batch, a2.layers = name, None, None, None
+            a2.no_e2e = args.no_e2e or name not in E2E_WORKLOADS
             o2 = run_ours(a2, rank, world, local_rank)
             r2 = o2["roofline"]
             out["other_workloads"][name] = {
                 "value": o2["value"], "unit": o2["unit"], "ms_per_step": o2["ms_per_step"], "steps": o2["steps"],
-                "config": o2["config"], "clocks": o2["clocks"],
-                "roofline": {k: r2[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic",
-                                                "bytes_per_launch", "kernel_ms_mean")},
+                "sequences_per_s": o2["sequences_per_s"], "config": o2["config"], "clocks": o2["clocks"],
+                "roofline": {k: r2[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "kernel",
+                                                "bytes_per_launch", "kernel_ms_mean", "launch_ms_from",
+                                                "kernel_ms_events", "frac_events")},
+                "gpu_launches": o2["gpu_launches"],
             }
-            if not args.no_unrolled and rank == 0:
+            for k in ("separate", "e2e"):
+                if k in o2:
+                    out["other_workloads"][name][k] = o2[k]
+            if not args.no_unrolled and rank == 0 and name in SIDE_WORKLOADS:
                 out["other_workloads"][name]["unrolled_baseline"] = unrolled_summary(o2, run_unrolled(name, local_rank))
-            if not args.no_accept and rank == 0:
+            if not args.no_accept and rank == 0 and name in SIDE_WORKLOADS:
                 out["other_workloads"][name]["accept_greedy"] = run_accept(name, args.vocab, local_rank)
     if rank == 0 and not args.no_unrolled:
         out["unrolled_baseline"] = unrolled_summary(out, run_unrolled(args.config, local_rank))

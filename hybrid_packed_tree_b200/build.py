@@ -1,6 +1,6 @@
 """Build ``libstree.so`` (the C ABI of include/stree.h) in-tree with nvcc for sm_100a.
 
-    python -m hybrid_packed_tree_b200.build [--force] [--debug]
+    python -m hybrid_packed_tree_b200.build [--force] [--verbose]
 
 The library is written next to this file so that it travels with the source
 tree; nothing is installed into site-packages.
@@ -36,16 +36,14 @@ def is_stale() -> bool:
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every .cu under csrc/ into libstree.so; returns its path."""
-    if not force and not debug and not is_stale():
+    if not force and not is_stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc, *ARCH, "-lineinfo", "-O3", "-std=c++17",
            "-cudart", "static", "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-o", tmp, *sources()]
-    if debug:
-        cmd.insert(1, "-DSTREE_DEBUG")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
@@ -56,10 +54,9 @@ def build(force: bool = False, debug: bool = False, verbose: bool = False) -> st
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--force", action="store_true")
-    ap.add_argument("--debug", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="pass -Xptxas=-v (registers, spills)")
     args = ap.parse_args(argv)
-    print(build(force=args.force, debug=args.debug, verbose=args.verbose))
+    print(build(force=args.force, verbose=args.verbose))
     return 0
 
 

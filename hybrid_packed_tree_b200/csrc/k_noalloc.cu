@@ -10,10 +10,15 @@
 // device array instead of a context's workspace.
 //
 // That array is a static __device__ object: every GPU that loads the library
-// holds its kNoAllocScratch bytes until the process exits.  Host code may not
-// pass the array's name to a kernel -- on the host it is only a stand-in -- so
-// the device address is looked up with cudaGetSymbolAddress, once per device,
-// with that device current, on the first call made on it.
+// holds its kNoAllocScratch bytes until the process exits (with lazy module
+// loading the array is placed on a device when the library's module is first
+// loaded there, at the latest by the first call of this entry point on it).
+// Host code may not pass the array's name to a kernel -- on the host it is only
+// a stand-in -- so the device address is looked up with cudaGetSymbolAddress,
+// with the device current, on the first call made on it; a call that finds a new
+// CUDA context on the device (after cudaDeviceReset) looks it up again.
+#include <cuda.h>
+
 #include <mutex>
 #include <string.h>
 
@@ -27,24 +32,62 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratch];
 
-std::mutex g_mutex;
-uint8_t *g_scratch[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Device address of the scratch on the current device (looked up once per device).
+struct ScratchSlot {
+    uint8_t *ptr = nullptr;
+    unsigned long long ctx_id = 0;
+};
+
+std::mutex g_mutex;
+ScratchSlot g_scratch[kMaxDevices];
+
+// Identifier of the current CUDA context; 0 when the thread has none yet, 1
+// when the driver cannot tell contexts apart (then the lookup is kept per device).
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (!get_current || !get_id) return 1;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of the scratch on the current device: looked up on the first
+// call on the device (with the device current) and again when the device has a
+// new context.
 cudaError_t scratch_address(uint8_t **out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const unsigned long long id = current_context_id();
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch[dev]) {
+    ScratchSlot &slot = g_scratch[dev];
+    if (!slot.ptr || id == 0 || slot.ctx_id != id) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
-        g_scratch[dev] = static_cast<uint8_t *>(p);
+        slot.ptr = static_cast<uint8_t *>(p);
+        slot.ctx_id = current_context_id();         // the lookup has made the context current
     }
-    *out = g_scratch[dev];
+    *out = slot.ptr;
     return cudaSuccess;
 }
 
@@ -73,15 +116,15 @@ extern "C" stree_status stree_tree_scan_commit_noalloc(
     a.maxlen = maxlen;
     a.h_new = h_new;
 
-    // Same shape rules as the context entry points.
+    // The shape rules and batch-0 behaviour of stree_tree_scan_commit.
     if (batch < 0 || n_nodes < 1 || nheads < 1 || ngroups < 1 || headdim < 1 || dstate < 1) return STREE_ERR_UNSUPPORTED;
+    if (batch == 0) return maxlen >= 0 ? STREE_OK : STREE_ERR_INVALID_ARG;
     if (n_nodes > kMaxNodes || headdim > kMaxDim || dstate > kMaxDim) return STREE_ERR_UNSUPPORTED;
     if (headdim % 8 != 0 || dstate % 8 != 0 || nheads % ngroups != 0 || nheads > 65535) return STREE_ERR_UNSUPPORTED;
     if (dtype != STREE_F32 && dtype != STREE_BF16) return STREE_ERR_UNSUPPORTED;
-    if (maxlen < 1) return STREE_ERR_INVALID_ARG;
-    if (batch == 0) return STREE_OK;
     if (!x || !dt || !A || !B || !C || !D || !h0 || !y || !parent || !accepted_path || !path_len || !h_new)
         return STREE_ERR_INVALID_ARG;
+    if (maxlen < 1) return STREE_ERR_INVALID_ARG;
     const void *ptrs[] = {x, dt, A, B, C, D, h0, y, h_new};
     for (const void *p : ptrs)
         if (!aligned16(p)) return STREE_ERR_MISALIGNED;
@@ -98,13 +141,14 @@ extern "C" stree_status stree_tree_scan_commit_noalloc(
     const size_t off_ok = off_depth + round256(nb * T * sizeof(int32_t));
     const size_t off_cb = off_ok + round256(nb * sizeof(int32_t));
     if (off_cb > kNoAllocScratch) return STREE_ERR_UNSUPPORTED;
-    // The tensor-core path's plan needs the device; look the scratch up first.
+    // The kernel choice needs the device; look the scratch up first.
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *base = nullptr;
     if (scratch_address(&base) != cudaSuccess) return STREE_ERR_CUDA;
-    const bool use_tc = tc_supported(a);
+    ScanPath path;
+    if (!select_path(STREE_KERNEL_AUTO, a, &path)) return STREE_ERR_UNSUPPORTED;
     size_t need = off_cb;
-    if (!use_tc) need += round256(nb * (size_t)ngroups * T * T * sizeof(float));
+    if (path == ScanPath::Simt) need += round256(nb * (size_t)ngroups * T * T * sizeof(float));
     if (need > kNoAllocScratch) return STREE_ERR_UNSUPPORTED;
 
     int32_t *err = err_out ? err_out : reinterpret_cast<int32_t *>(base + off_err);
@@ -114,17 +158,18 @@ extern "C" stree_status stree_tree_scan_commit_noalloc(
     // The error word must start at zero; masks, depths, flags and the pair
     // scratch are fully rewritten by the kernels below.
     if (cudaMemsetAsync(err, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return STREE_ERR_CUDA;
-    if (launch_build_tree(parent, n_nodes, batch, anc, depth, ok, err, s) != cudaSuccess) return STREE_ERR_CUDA;
     a.tree.anc = anc;
     a.tree.depth = depth;
     a.tree.ok = ok;
     a.tree.T = n_nodes;
     a.tree.W = (int)W;
     a.tree.batch = batch;
-    a.parent = parent;                       // the builder was launched right before
+    a.parent = parent;                       // the launch rebuilds the tree into the scratch
+    a.tree_anc = anc;
+    a.tree_depth = depth;
+    a.tree_ok = ok;
     a.err = err;
-    if (use_tc) return launch_scan_tc(a, s) == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
-    a.cb = reinterpret_cast<float *>(base + off_cb);
-    if (launch_cb_pairs(a, s) != cudaSuccess) return STREE_ERR_CUDA;
-    return launch_scan_simt(a, s) == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
+    if (path == ScanPath::Simt) a.cb = reinterpret_cast<float *>(base + off_cb);
+    int64_t launches = 0;
+    return launch_scan(path, a, s, &launches) == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
 }

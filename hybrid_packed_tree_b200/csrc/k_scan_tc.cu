@@ -64,11 +64,12 @@ enum Misc { M_TMEM = 0, M_ABORT, M_LEN, M_STATE, M_INSMEM, M_TOTAL, M_OK, M_DTK,
             kMiscWords = M_WSUM + kWarps };
 // mbarriers: TMA stage full / epilogue done with a stage (ring of S), tensor-memory
 // accumulator full / empty (ring of 2), masked-decay matrix full / empty,
-// per-tile coefficients full / empty (ring of 2), and for the tensor-core commit
-// its coefficient operand written and its (single) product read.
+// per-tile coefficients full / empty (ring of 2), for the tensor-core commit its
+// coefficient operand written and its (single) product read, and the MMA drain
+// after an abort.
 enum Bars { B_FULL = 0, B_EPID = kMaxStages, B_ACCF = 2 * kMaxStages, B_ACCE = B_ACCF + 2, B_MHF = B_ACCE + 2,
             B_MHE = B_MHF + 1, B_COEFF = B_MHE + 1, B_COEFE = B_COEFF + 2, B_CFF = B_COEFE + 2, B_CME = B_CFF + 1,
-            kNumBars = B_CME + 1 };
+            B_DRAIN = B_CME + 1, kNumBars = B_DRAIN + 1 };
 
 struct TcParams {
     const __nv_bfloat16 *__restrict__ dt;
@@ -80,7 +81,11 @@ struct TcParams {
     const int32_t *__restrict__ path_len;
     const int32_t *__restrict__ parent;    // non-NULL: masks built in-kernel, inputs complete at launch
     TreeView tree;
+    uint32_t *tree_anc;                    // with parent: the tree written here for later calls (or NULL)
+    int32_t *tree_depth, *tree_ok;
     int32_t *err;
+    unsigned long long wait_ns;            // limit of every bounded wait
+    int fault;                             // test hook: 1 withholds the first tile's coefficient hand-off
     int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, pre, bs_mh, tc_commit, hpt, pair_cap,
         acc_cols, cm_col;
     uint32_t tmem_cols;
@@ -278,19 +283,6 @@ __device__ __forceinline__ uint32_t k8_off(int row, int k)
     return (uint32_t)(row >> 3) * 256u + (uint32_t)(k >> 2) * 128u + (uint32_t)(row & 7) * 16u + (uint32_t)(k & 3) * 4u;
 }
 
-#ifdef STREE_TRACE
-// Profiling builds only: wall-clock stamps of pipeline events for four CTAs.
-__device__ unsigned long long g_trace[4 * 32 * 24];
-__device__ __forceinline__ void trace_event(uint32_t k, int ev)
-{
-    const int slot = blockIdx.x == 0 ? 0 : blockIdx.x == 37 ? 1 : blockIdx.x == 74 ? 2 : blockIdx.x == 111 ? 3 : -1;
-    if (slot >= 0 && k < 32) g_trace[(slot * 32 + k) * 24 + ev] = ptx::globaltimer();
-}
-#define STREE_TR(k, ev) trace_event((k), (ev))
-#else
-#define STREE_TR(k, ev) ((void)0)
-#endif
-
 // Eight 32-bit shared-memory loads issued back to back (addresses in the shared window).
 __device__ __forceinline__ void lds_f32x8(const uint32_t (&a)[8], float (&v)[8])
 {
@@ -378,14 +370,12 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     };
     auto bar = [&](int i) { return ptx::smem_u32(&bars[i]); };
 
-    if (tid == 0) STREE_TR(31, 0);
     const uint32_t h0_stage_bytes = (uint32_t)RB * 512u;
     const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u;
     const int start = (int)((long long)blockIdx.x * p.ntiles / gridDim.x);
     const int end = (int)((long long)(blockIdx.x + 1) * p.ntiles / gridDim.x);
-    // With p.pre every input is complete at launch (the preceding launch is the
-    // tree builder, which started after all earlier work): the first S tiles are
-    // requested before anything else.
+    // With p.pre the first S tiles are requested before anything else, once the
+    // preceding grid (the kernel is a programmatic dependent) has completed.
     const uint32_t npre = p.pre ? (uint32_t)min(S, end - start) : 0u;
     uint32_t loads_issued = 0, stores_issued = 0;
 
@@ -393,7 +383,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     // every wait returns false at once and no role does further work.
     auto wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
         if (misc[M_ABORT]) return false;
-        if (ptx::mbar_wait(b, parity)) return true;
+        if (ptx::mbar_wait(b, parity, p.wait_ns)) return true;
         latch_error(p.err, STREE_ERR_TIMEOUT, blockIdx.x, where, (int)parity);
         misc[M_ABORT] = 1;
         return false;
@@ -412,7 +402,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         if (what & 2) ptx::tma_store_3d(&tm_hn, 0, b * HP + r0, 0, ptx::smem_u32(h0s + s * h0_stage_bytes));
         ptx::bulk_commit();
         stores_issued = q + 1;
-        STREE_TR(q, 10);
     };
     // Producer: TMA loads of tile k into stage k % S once tile k - S has left it.
     auto produce = [&](uint32_t k, int t) {
@@ -420,7 +409,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         if (k >= (uint32_t)S) {
             store_tile(k - S);
             ptx::bulk_wait_read_all();
-            STREE_TR(k - S, 11);
         }
         if (misc[M_ABORT]) return;
         const int b = t / p.tps, r0 = (t % p.tps) * RB;
@@ -431,9 +419,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         const uint32_t xdst = ptx::smem_u32(xs + s * p.x_stage);
         for (int nb = 0; nb < p.NB; ++nb) ptx::tma_load_2d(xdst + nb * xbs, &tm_x, r0 + nb * 64, b * T, fb);
         loads_issued = k + 1;
-        STREE_TR(k, 0);
     };
 
+    if (p.pre) asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) {
         ptx::prefetch_tensormap(&tm_h0);
         ptx::prefetch_tensormap(&tm_x);
@@ -453,6 +441,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
         ptx::mbar_init(bar(B_MHE), 1);
         ptx::mbar_init(bar(B_CFF), kPrepThreads);
         ptx::mbar_init(bar(B_CME), kEpiWarps);
+        ptx::mbar_init(bar(B_DRAIN), 1);
         ptx::fence_mbar_init();
         for (int q = 0; q < kMiscWords; ++q) misc[q] = 0;
         for (uint32_t q = 0; q < npre; ++q) produce(q, start + (int)q);
@@ -471,7 +460,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     // launch: nothing global is read before it has completed.
     if (!p.pre) asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();                                  // misc cleared before the allocation writes it
-    if (tid == 0) STREE_TR(31, 1);
     if (warp == kMmaWarp) {
         ptx::tmem_alloc(ptx::smem_u32(const_cast<int32_t *>(&misc[M_TMEM])), p.tmem_cols);
         ptx::tmem_relinquish();
@@ -481,7 +469,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = static_cast<uint32_t>(misc[M_TMEM]);
-    if (tid == 0) STREE_TR(31, 2);
 
     int cur_key = -1, cur_b = -1;
     // Prep warps: dt of the next tile, requested while the current one is prepared.
@@ -506,9 +493,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             if (warp == kProducerWarp && lane == 0 && !produced) produce(k, t);   // keep the stream going
             produced = true;
             __syncthreads();                                   // every earlier tile is consumed
-            if (tid == 0) STREE_TR(k, 12);
             const bool new_b = (b != cur_b);
-            [[maybe_unused]] const uint32_t swrow = cur_key < 0 ? 30u : 29u;   // trace row of this switch
             // Phase 1: every global read of this (sequence, group) in flight at once:
             // asynchronous copies for the B rows, parent, path, A and D (or the
             // context's tree), plain loads for dt and C (C is widened to fp32).
@@ -580,7 +565,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             ptx::cp_async_wait_all();
             __syncthreads();
-            if (tid == 0) STREE_TR(swrow, 0);
             if (new_b) {
                 bool okb;
                 if (p.parent) {
@@ -607,6 +591,24 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     if (tid == 0) misc[M_OK] = okb;
                     __syncthreads();
+                    if (t % p.tps == 0) {
+                        // The CTA holding the sequence's first tile keeps its tree for
+                        // later calls and reports an invalid one (first bad node).
+                        if (p.tree_anc)
+                            for (int q = tid; q < T * W; q += kThreads) p.tree_anc[(size_t)b * T * W + q] = ancs[q];
+                        if (p.tree_depth)
+                            for (int i = tid; i < T; i += kThreads) p.tree_depth[(size_t)b * T + i] = dep[i];
+                        if (tid == 0) {
+                            if (p.tree_ok) p.tree_ok[b] = okb ? 1 : 0;
+                            for (int i = 0; i < T && !okb; ++i) {
+                                const int v = par[i];
+                                if ((i == 0) ? (v != -1) : (v < 0 || v >= i)) {
+                                    latch_error(p.err, STREE_ERR_BAD_TREE, b, i, v);
+                                    break;
+                                }
+                            }
+                        }
+                    }
                 } else {
                     okb = misc[M_OK] != 0;
                 }
@@ -662,7 +664,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 cur_b = b;
             }
             __syncthreads();
-            if (tid == 0) STREE_TR(swrow, 1);
             // Phase 3: path rows of B (fp32) for the commit, C_i . B_j of every ancestor pair.
             if (misc[M_STATE] && p.tc_commit && misc[M_LEN] <= kPathRows) {
                 // B^T of the path rows, K-major fp32 (zeros past the path), for the commit MMA.
@@ -692,7 +693,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             if (misc[M_INSMEM]) {
                 const int total = misc[M_TOTAL];
-                if (tid == 0) STREE_TR(swrow, 2);
                 // Node i's pairs: its ancestors in increasing order.
                 for (int i = tid; i < T; i += kThreads) {
                     int q = poff[i];
@@ -707,7 +707,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                 }
                 __syncthreads();
-                if (tid == 0) STREE_TR(swrow, 3);
                 // Four lanes per pair, a quarter of the state columns each.
                 const int part = lane & 3;
                 for (int q0 = (tid >> 2); q0 < ((total + 7) & ~7); q0 += kThreads / 4) {
@@ -721,7 +720,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     if (part == 0 && q0 < total) pcb[q] = v;
                 }
             }
-            if (tid == 0) STREE_TR(swrow, 4);
             if (p.bs_mh) {                                     // B rows read: clear the region for M_h
                 __syncthreads();
                 for (uint32_t o = tid * 16u; o < (uint32_t)hpt * p.mh_head; o += kThreads * 16u)
@@ -729,7 +727,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             }
             ptx::fence_proxy_async_smem();
             __syncthreads();
-            if (tid == 0) STREE_TR(k, 13);
             cur_key = key;
         }
         const int len = misc[M_LEN];
@@ -748,7 +745,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 const uint32_t acc = tmem + (uint32_t)(a * p.acc_cols);
                 bool ok = wait(bar(B_FULL + s), sph, 20);
                 if (ok && k >= 2) ok = wait(bar(B_ACCE + a), ((k >> 1) - 1) & 1, 21);
-                STREE_TR(k, 1);
                 if (ok) {
                     ptx::tc_fence_after();
                     const uint32_t a0 = ptx::smem_u32(h0t), b0 = ptx::smem_u32(cs);
@@ -761,7 +757,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                                           ptx::desc_kmajor_sw128(b0 + kb * T_pad * 128 + kk * 32), idesc_root,
                                           (kb | kk) != 0);
                     ok = wait(bar(B_MHF), k & 1, 22);
-                    STREE_TR(k, 2);
                 }
                 if (ok) {
                     ptx::tc_fence_after();
@@ -793,7 +788,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                         ptx::mma_commit(bar(B_ACCF + a));
                         ptx::mma_commit(bar(B_MHE));
                     }
-                    STREE_TR(k, 3);
                 }
                 if (tcc) ++ncm;
             }
@@ -809,7 +803,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             bool ok = !misc[M_ABORT];
             float *dts = coef(c, 0), *Ls = coef(c, 1), *eLs = coef(c, 2), *wts = coef(c, 3);
             float *alpha = coef(c, 4);
-            if (ptid == 0) STREE_TR(k, 4);
             if (ok && misc[M_DTK] != (int)k + 1) {             // not already read by the switch
                 if (dnext_k == (int)k) {
 #pragma unroll
@@ -851,8 +844,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     if (ptid < hpt) alpha[ptid] = len > 0 ? eLs[ptid * T + leaf] : 1.f;
                 }
-                mbar_arrive(bar(B_COEFF + c));
-                if (ptid == 0) STREE_TR(k, 5);
+                // (The failure-path test hook withholds this arrival for the first
+                // tile, so that the epilogue's bounded wait runs out.)
+                if (!(p.fault == 1 && k == 0)) mbar_arrive(bar(B_COEFF + c));
                 // Masked decay matrix of every head of the tile (bf16, K-major swizzled):
                 // M_h[i][j] = exp(L_i - L_j) (C_i . B_j) dt_j for j an ancestor-or-self of i,
                 // plus D_h on the diagonal, so that the tree MMA also yields the skip term.
@@ -884,7 +878,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     ptx::fence_proxy_async_smem();
                     mbar_arrive(bar(B_MHF));
-                    if (ptid == 0) STREE_TR(k, 6);
                     // dt of the next tile when it belongs to the same (sequence, group)
                     // (a switch reads its own); hpt * T <= 512 values.
                     const int t1 = t + 1, b1 = t1 / p.tps, hf1 = (t1 % p.tps) * RB / P;
@@ -937,7 +930,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
             named_sync(kBarEpi, kEpiThreads);
             // Warp-uniform decision (tcgen05.ld below is a warp-collective instruction).
             const bool run = __all_sync(0xffffffffu, !misc[M_ABORT]);
-            if (etid == 0) STREE_TR(k, 7);
             if (run) ptx::tc_fence_after();
             const float *eLs = coef(c, 2), *wts = coef(c, 3), *alpha = coef(c, 4);
             if (run && commit && !tcc) {
@@ -946,15 +938,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 const int hh = (r0 + row) / P - hfirst;
                 const MnCol xc(row, xbs);
                 const int cols = kDstate / tpr;
-                if (warp == 8 && lane == 0) STREE_TR(k, 20);
                 for (int c_lo = part * cols; c_lo < (part + 1) * cols; c_lo += 32)
                     commit_rows<32>(h0t, xt, xc, Bp, p.tc_commit ? 0 : kPathRows, Bseq, brow, pnode, wts + hh * T,
                                     alpha[hh], len, RB, row, c_lo);
-                if (warp == 8 && lane == 0) STREE_TR(k, 21);
             }
-            if (warp == 8 && lane == 0) STREE_TR(k, 19);
             named_sync(kBarEpi, kEpiThreads);                  // x rows of the path are read
-            if (etid == 0) STREE_TR(k, 8);
             // A warp reads only its own quarter of the tensor-memory lanes: 32 * (warp % 4).
             // M = 128 puts tile row r in lane r; M = 64 puts rows 16q..16q+15 in
             // lanes 32q..32q+15, so every quarter (and every SM sub-partition) gets rows.
@@ -1020,7 +1008,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                 }
             }
-            if (warp == 8 && lane == 0) STREE_TR(k, 16);
             if (tcc && run) {
                 // h_new = alpha h0 + D, D read from tensor memory (same lane mapping as y).
                 {
@@ -1064,10 +1051,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 mbar_arrive(bar(B_COEFE + c));
             }
             ptx::fence_proxy_async_smem();
-            if (warp == 8 && lane == 0) STREE_TR(k, 17);
-            if (warp == 6 && lane == 0) STREE_TR(k, 18);
             named_sync(kBarEpi, kEpiThreads);
-            if (etid == 0) STREE_TR(k, 9);
             if (run && etid == 0) {
                 misc[M_SDESC + 2 * s] = t;                     // the producer issues the stores
                 misc[M_SDESC + 2 * s + 1] = (misc[M_OK] ? 1 : 0) | (commit ? 2 : 0);
@@ -1077,11 +1061,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     }
 
     // ---------------------------------------------------------------- teardown
-    if (tid == 0) STREE_TR(31, 4);
     if (warp == kProducerWarp && lane == 0) {
         for (uint32_t q = stores_issued; q < k && !misc[M_ABORT]; ++q) store_tile(q);
         ptx::bulk_wait_all();
-        STREE_TR(31, 6);
         if (misc[M_ABORT]) {
             // Loads issued but never consumed may still land in this CTA's shared
             // memory: give them a bounded wait before the CTA exits.
@@ -1089,16 +1071,18 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 ptx::mbar_wait(bar(B_FULL + q % S), (q / S) & 1);
         }
     }
+    if (warp == kMmaWarp && lane == 0 && misc[M_ABORT]) {
+        // After an abort some issued MMAs may have no commit: wait (bounded) until
+        // every MMA of this thread has completed before the tensor memory is freed.
+        ptx::mma_commit(bar(B_DRAIN));
+        ptx::mbar_wait(bar(B_DRAIN), 0);
+    }
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, p.tmem_cols);
-        if (lane == 0) STREE_TR(31, 5);
     }
-    // The grid completes no earlier than the launch it depends on (the tree
-    // builder), so later work on the stream sees both.
-    if (p.pre) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------------- host side
@@ -1347,6 +1331,11 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     p.parent = a.parent;
     p.pre = a.parent != nullptr;
     p.tree = a.tree;
+    p.tree_anc = a.tree_anc;
+    p.tree_depth = a.tree_depth;
+    p.tree_ok = a.tree_ok;
+    p.wait_ns = a.wait_ns ? a.wait_ns : ptx::kWaitLimitNs;
+    p.fault = a.fault;
     p.err = a.err;
 
     EncodeTiledFn enc = encode_fn();
@@ -1388,9 +1377,10 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     // 512 threads at 128 registers leave room for one CTA per SM.
     long long grid = num_sms();
     if (grid > p.ntiles) grid = p.ntiles;
-    // Programmatic dependent launch.  After the tree builder (parent given) the
-    // kernel needs nothing it writes and overlaps it entirely; otherwise the
-    // prologue (barriers, tensor memory) overlaps the tail of the preceding kernel.
+    // Programmatic dependent launch: the kernel waits for the preceding grid
+    // before its first global read (at entry with parent[] given, after the
+    // barrier and tensor-memory set-up otherwise), so that much overlaps the
+    // preceding grid's tail.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
@@ -1405,15 +1395,3 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
 }
 
 }  // namespace stree
-
-#ifdef STREE_TRACE
-extern "C" int stree_debug_trace(unsigned long long *host, size_t n)
-{
-    return (int)cudaMemcpyFromSymbol(host, stree::g_trace, n * sizeof(unsigned long long));
-}
-extern "C" int stree_debug_trace_clear(void)
-{
-    static unsigned long long zero[4 * 32 * 24];
-    return (int)cudaMemcpyToSymbol(stree::g_trace, zero, sizeof(zero));
-}
-#endif

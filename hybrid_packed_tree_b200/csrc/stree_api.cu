@@ -25,6 +25,9 @@ struct stree_ctx {
     bool has_scan = false;
     ScanArgs last{};
     int64_t launches = 0;
+    stree_kernel last_kernel = STREE_KERNEL_AUTO;   // the kernel of the last scan (AUTO: none yet)
+    unsigned long long wait_ns = 0;                 // bounded-wait limit (0: the kernel's default)
+    int fault = 0;                                  // failure-path test hook
 };
 
 namespace {
@@ -60,7 +63,9 @@ TreeView tree_view(const stree_ctx *c)
     return tv;
 }
 
-stree_status build_into_ctx(stree_ctx *c, const int32_t *parent, int T, int batch, cudaStream_t s)
+// Sizes the context's tree workspace for (T, batch) and records them; nothing is
+// launched (the scan kernels or the tree builder fill it).
+stree_status ensure_tree(stree_ctx *c, const int32_t *parent, int T, int batch)
 {
     if (T < 1 || T > kMaxNodes || batch < 0) return STREE_ERR_UNSUPPORTED;
     if (!parent && batch > 0) return STREE_ERR_INVALID_ARG;
@@ -73,6 +78,13 @@ stree_status build_into_ctx(stree_ctx *c, const int32_t *parent, int T, int batc
     if ((st = ensure(&c->ok, &c->cap_batch, nb)) != STREE_OK) return st;
     c->tree_T = T;
     c->tree_batch = batch;
+    return STREE_OK;
+}
+
+stree_status build_into_ctx(stree_ctx *c, const int32_t *parent, int T, int batch, cudaStream_t s)
+{
+    stree_status st = ensure_tree(c, parent, T, batch);
+    if (st != STREE_OK) return st;
     if (batch > 0) ++c->launches;
     return cuda_status(launch_build_tree(parent, T, batch, c->anc, c->depth, c->ok, c->err, s));
 }
@@ -104,30 +116,32 @@ stree_status check_commit_args(const int32_t *path, const int32_t *path_len, int
     return STREE_OK;
 }
 
-// Runs the scan (and the commit, when a.path is set) for a tree already in the ctx.
+// Runs the scan (and the fused commit when a.path is set).  With a.parent set the
+// tree is rebuilt into the context by the launch; otherwise the context's tree is used.
 stree_status run_scan(stree_ctx *c, ScanArgs &a, cudaStream_t s)
 {
     if (c->tree_batch != a.batch || c->tree_T != a.T) return STREE_ERR_NO_TREE;
     a.tree = tree_view(c);
     a.err = c->err;
+    a.wait_ns = c->wait_ns;
+    a.fault = c->fault;
+    if (a.parent) {
+        a.tree_anc = c->anc;
+        a.tree_depth = c->depth;
+        a.tree_ok = c->ok;
+    }
     if (a.batch == 0) return STREE_OK;
-    bool use_tc = false;
-    if (c->kernel == STREE_KERNEL_TC) {
-        if (!tc_supported(a)) return STREE_ERR_UNSUPPORTED;
-        use_tc = true;
-    } else if (c->kernel == STREE_KERNEL_AUTO) {
-        use_tc = tc_supported(a);
+    ScanPath path;
+    if (!select_path(c->kernel, a, &path)) return STREE_ERR_UNSUPPORTED;
+    c->last_kernel = path == ScanPath::Small ? STREE_KERNEL_SMALL
+                     : path == ScanPath::Tc  ? STREE_KERNEL_TC
+                                             : STREE_KERNEL_SIMT;
+    if (path == ScanPath::Simt) {
+        stree_status st = ensure(&c->cb, &c->cap_cb, (size_t)a.batch * a.G * a.T * a.T);
+        if (st != STREE_OK) return st;
+        a.cb = c->cb;
     }
-    ++c->launches;
-    if (use_tc) return cuda_status(launch_scan_tc(a, s));     // computes C.B pairs itself
-    stree_status st = ensure(&c->cb, &c->cap_cb, (size_t)a.batch * a.G * a.T * a.T);
-    if (st != STREE_OK) return st;
-    a.cb = c->cb;
-    if (a.y) {
-        ++c->launches;
-        if ((st = cuda_status(launch_cb_pairs(a, s))) != STREE_OK) return st;
-    }
-    return cuda_status(launch_scan_simt(a, s));
+    return cuda_status(launch_scan(path, a, s, &c->launches));
 }
 
 ScanArgs make_args(const void *x, const void *dt, const float *A, const void *B, const void *C,
@@ -143,6 +157,70 @@ ScanArgs make_args(const void *x, const void *dt, const float *A, const void *B,
 }
 
 }  // namespace
+
+namespace stree {
+
+// Batches up to this many state rows (batch x nheads x headdim) take the
+// small-batch kernel when both it and the tensor-core kernel support the shape:
+// below it a launch is bound by latency, which the small kernel's short chain
+// serves better than the tensor-core pipeline.
+constexpr long long kSmallRows = 65536;
+
+bool select_path(stree_kernel sel, const ScanArgs &a, ScanPath *out)
+{
+    switch (sel) {
+    case STREE_KERNEL_SIMT:
+        *out = ScanPath::Simt;
+        return true;
+    case STREE_KERNEL_TC:
+        if (!tc_supported(a)) return false;
+        *out = ScanPath::Tc;
+        return true;
+    case STREE_KERNEL_SMALL:
+        if (!small_supported(a)) return false;
+        *out = ScanPath::Small;
+        return true;
+    case STREE_KERNEL_AUTO: {
+        const bool small = small_supported(a), tc = tc_supported(a);
+        const long long rows = (long long)a.batch * a.H * a.P;
+        if (small && (!tc || rows <= kSmallRows)) *out = ScanPath::Small;
+        else if (tc) *out = ScanPath::Tc;
+        else *out = ScanPath::Simt;
+        return true;
+    }
+    }
+    return false;
+}
+
+cudaError_t launch_scan(ScanPath path, const ScanArgs &a, cudaStream_t s, int64_t *launches)
+{
+    if (a.batch == 0) return cudaSuccess;
+    cudaError_t e;
+    switch (path) {
+    case ScanPath::Small:
+        ++*launches;
+        return launch_scan_small(a, s);
+    case ScanPath::Tc:
+        ++*launches;
+        return launch_scan_tc(a, s);
+    case ScanPath::Simt:
+        if (a.parent) {
+            ++*launches;
+            if ((e = launch_build_tree(a.parent, a.T, a.batch, a.tree_anc, a.tree_depth, a.tree_ok, a.err, s)) !=
+                cudaSuccess)
+                return e;
+        }
+        if (a.y) {
+            ++*launches;
+            if ((e = launch_cb_pairs(a, s)) != cudaSuccess) return e;
+        }
+        ++*launches;
+        return launch_scan_simt(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace stree
 
 extern "C" {
 
@@ -179,7 +257,8 @@ stree_status stree_ctx_destroy(stree_ctx *c)
 stree_status stree_ctx_set_kernel(stree_ctx *c, stree_kernel k)
 {
     if (!c) return STREE_ERR_INVALID_ARG;
-    if (k != STREE_KERNEL_AUTO && k != STREE_KERNEL_SIMT && k != STREE_KERNEL_TC) return STREE_ERR_INVALID_ARG;
+    if (k != STREE_KERNEL_AUTO && k != STREE_KERNEL_SIMT && k != STREE_KERNEL_TC && k != STREE_KERNEL_SMALL)
+        return STREE_ERR_INVALID_ARG;
     c->kernel = k;
     return STREE_OK;
 }
@@ -188,6 +267,27 @@ stree_status stree_ctx_launch_count(stree_ctx *c, int64_t *count)
 {
     if (!c || !count) return STREE_ERR_INVALID_ARG;
     *count = c->launches;
+    return STREE_OK;
+}
+
+stree_status stree_ctx_set_wait_limit(stree_ctx *c, uint64_t ns)
+{
+    if (!c) return STREE_ERR_INVALID_ARG;
+    c->wait_ns = ns;
+    return STREE_OK;
+}
+
+stree_status stree_ctx_set_test_fault(stree_ctx *c, int fault)
+{
+    if (!c || fault < 0 || fault > 1) return STREE_ERR_INVALID_ARG;
+    c->fault = fault;
+    return STREE_OK;
+}
+
+stree_status stree_ctx_last_kernel(stree_ctx *c, stree_kernel *kernel)
+{
+    if (!c || !kernel) return STREE_ERR_INVALID_ARG;
+    *kernel = c->last_kernel;
     return STREE_OK;
 }
 
@@ -221,9 +321,9 @@ stree_status stree_tree_scan(stree_ctx *c, const void *x, const void *dt, const 
     stree_status st = check_scan_args(a);
     if (st != STREE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((parent || batch == 0) && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
+    if ((parent || batch == 0) && (st = ensure_tree(c, parent, n_nodes, batch)) != STREE_OK) return st;
     ScanArgs rec = a;
-    a.parent = parent;                      // the builder was launched right before
+    a.parent = parent;                      // the launch rebuilds the context's tree
     if ((st = run_scan(c, a, s)) != STREE_OK) return st;
     c->last = rec;
     c->has_scan = true;
@@ -248,6 +348,7 @@ stree_status stree_commit(stree_ctx *c, const int32_t *path, const int32_t *path
     a.err = c->err;
     if (a.batch == 0) return STREE_OK;
     ++c->launches;
+    if (commit_supported(a)) return cuda_status(launch_commit(a, static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_scan_simt(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -264,9 +365,9 @@ stree_status stree_tree_scan_commit(stree_ctx *c, const void *x, const void *dt,
     if (st != STREE_OK) return st;
     if ((st = check_commit_args(path, path_len, maxlen, h_new, batch)) != STREE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((parent || batch == 0) && (st = build_into_ctx(c, parent, n_nodes, batch, s)) != STREE_OK) return st;
+    if ((parent || batch == 0) && (st = ensure_tree(c, parent, n_nodes, batch)) != STREE_OK) return st;
     ScanArgs rec = a;
-    a.parent = parent;                      // the builder was launched right before
+    a.parent = parent;                      // the launch rebuilds the context's tree
     a.path = path;
     a.path_len = path_len;
     a.maxlen = maxlen;

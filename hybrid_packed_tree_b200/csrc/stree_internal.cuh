@@ -43,13 +43,21 @@ struct ScanArgs {
     int maxlen;
     float *h_new;
     TreeView tree;
-    // Set only when the tree builder was launched on the same stream right before
-    // the scan: the tensor-core kernel then builds the masks itself from parent[]
-    // and may read every input before that launch has finished.
+    // Set when the call passes the tree: the small-batch and tensor-core kernels
+    // then build the masks themselves from parent[] and write them (masks, depths,
+    // flags, the same layouts as TreeView) to the tree_* arrays for later calls;
+    // the CUDA-core path has the tree builder write them first.
     const int32_t *parent;
+    uint32_t *tree_anc;
+    int32_t *tree_depth, *tree_ok;
     float *cb;                         // scratch [batch, G, T, T]: C_i . B_j on ancestor pairs
     int32_t *err;
+    unsigned long long wait_ns;        // tensor-core kernel: bounded-wait limit (0: the default)
+    int fault;                         // tensor-core kernel: failure-path test hook (0: off)
 };
+
+// The kernels that can run a scan.
+enum class ScanPath { Small, Tc, Simt };
 
 // Kernel launchers (each returns cudaSuccess or the launch error).
 cudaError_t launch_build_tree(const int32_t *parent, int T, int batch, uint32_t *anc, int32_t *depth,
@@ -62,6 +70,23 @@ cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t s);
 // Tensor-core path: whether the shape is supported, and the launcher.
 bool tc_supported(const ScanArgs &a);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
+
+// Small-batch path: whether the shape is supported, and the launcher.
+bool small_supported(const ScanArgs &a);
+cudaError_t launch_scan_small(const ScanArgs &a, cudaStream_t s);
+
+// Commit by replay of the accepted path alone (no tree term, no root term).
+bool commit_supported(const ScanArgs &a);
+cudaError_t launch_commit(const ScanArgs &a, cudaStream_t s);
+
+// Resolves a kernel selection against the shape; false when the selection
+// cannot run it (STREE_ERR_UNSUPPORTED).
+bool select_path(stree_kernel sel, const ScanArgs &a, ScanPath *out);
+
+// Launches the scan (and the fused commit when a.path is set) on `path`.  With
+// a.parent set the tree is rebuilt into a.tree_*; the CUDA-core path needs a.cb.
+// *launches is increased by the number of kernels launched.
+cudaError_t launch_scan(ScanPath path, const ScanArgs &a, cudaStream_t s, int64_t *launches);
 
 __device__ __forceinline__ float load_as_float(const void *p, size_t i, stree_dtype dt)
 {

@@ -32,11 +32,12 @@ STATUS_NAMES = {
     8: "STREE_ERR_NO_TREE",
 }
 STREE_F32, STREE_BF16 = 0, 1
-KERNELS = {"auto": 0, "simt": 1, "tc": 2}
+KERNELS = {"auto": 0, "simt": 1, "tc": 2, "small": 3}
 
 # Every exported symbol of include/stree.h.
 EXPORTS = (
     "stree_ctx_create", "stree_ctx_destroy", "stree_ctx_set_kernel", "stree_ctx_launch_count",
+    "stree_ctx_last_kernel", "stree_ctx_set_wait_limit", "stree_ctx_set_test_fault",
     "stree_build_tree",
     "stree_tree_scan", "stree_commit", "stree_tree_scan_commit", "stree_tree_scan_commit_noalloc",
     "stree_resolve_path", "stree_unrolled_scan", "stree_accept_greedy",
@@ -48,6 +49,9 @@ _lib.stree_ctx_create.argtypes = [ctypes.POINTER(_vp)]
 _lib.stree_ctx_destroy.argtypes = [_vp]
 _lib.stree_ctx_set_kernel.argtypes = [_vp, _i]
 _lib.stree_ctx_launch_count.argtypes = [_vp, ctypes.POINTER(ctypes.c_int64)]
+_lib.stree_ctx_last_kernel.argtypes = [_vp, ctypes.POINTER(ctypes.c_int)]
+_lib.stree_ctx_set_wait_limit.argtypes = [_vp, ctypes.c_uint64]
+_lib.stree_ctx_set_test_fault.argtypes = [_vp, _i]
 _lib.stree_build_tree.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp]
 _lib.stree_tree_scan.argtypes = [_vp] * 9 + [_i] * 7 + [_vp, _vp]
 _lib.stree_commit.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
@@ -155,6 +159,23 @@ def stree_ctx_launch_count(ctx: Ctx) -> int:
     n = ctypes.c_int64(0)
     _check(_lib.stree_ctx_launch_count(ctx.handle, ctypes.byref(n)), "stree_ctx_launch_count")
     return int(n.value)
+
+
+def stree_ctx_last_kernel(ctx: Ctx) -> str:
+    """Name ("simt", "tc" or "small") of the kernel that ran the last scan; "auto" before any."""
+    k = ctypes.c_int(0)
+    _check(_lib.stree_ctx_last_kernel(ctx.handle, ctypes.byref(k)), "stree_ctx_last_kernel")
+    return {v: n for n, v in KERNELS.items()}[int(k.value)]
+
+
+def stree_ctx_set_wait_limit(ctx: Ctx, ns: int = 0):
+    """Bounded-wait limit of the tensor-core kernel in ns (0: the default, about 1 s)."""
+    _check(_lib.stree_ctx_set_wait_limit(ctx.handle, int(ns)), "stree_ctx_set_wait_limit")
+
+
+def stree_ctx_set_test_fault(ctx: Ctx, fault: int = 0):
+    """Failure-path test hook: 1 makes a bounded wait of the tensor-core kernel run out."""
+    _check(_lib.stree_ctx_set_test_fault(ctx.handle, int(fault)), "stree_ctx_set_test_fault")
 
 
 def stree_build_tree(ctx: Ctx, parent, anc_out=None, depth_out=None, stream=None):

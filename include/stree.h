@@ -42,12 +42,12 @@
  * of 8 in [8, 256], nheads a multiple of ngroups.  Pointers to tensors must be
  * 16-byte aligned.  batch = 0 is a no-op that returns STREE_OK.
  *
- * Precision: all accumulation is fp32.  The CUDA-core kernel (STREE_KERNEL_SIMT,
- * and every fp32 input) computes in fp32 throughout.  The tensor-core kernel
- * (bf16 inputs, dstate 128, n_nodes <= 128, headdim a multiple of 32) rounds h0 to
- * tf32 in the root term, the masked decay matrix (D_h on its diagonal included) to
- * bf16, and the commit coefficients dt-weighted x to tf32; each rounding is below
- * the bf16 rounding of y itself.
+ * Precision: all accumulation is fp32.  The CUDA-core kernels (STREE_KERNEL_SIMT
+ * and STREE_KERNEL_SMALL, and every fp32 input) compute in fp32 throughout.  The
+ * tensor-core kernel (bf16 inputs, dstate 128, n_nodes <= 128, headdim a multiple
+ * of 32) rounds h0 to tf32 in the root term, the masked decay matrix (D_h on its
+ * diagonal included) to bf16, and the commit coefficients dt-weighted x to tf32;
+ * each rounding is below the bf16 rounding of y itself.
  *
  * Ownership and threading: the caller owns every tensor.  A context (stree_ctx)
  * owns the library's device workspace (tree masks, depths, per-sequence flags,
@@ -91,9 +91,12 @@ typedef enum { STREE_F32 = 0, STREE_BF16 = 1 } stree_dtype;
 
 /* Which scan kernel a context uses (stree_ctx_set_kernel). */
 typedef enum {
-    STREE_KERNEL_AUTO = 0,      /* tensor-core kernel where supported, else SIMT */
+    STREE_KERNEL_AUTO = 0,      /* SMALL for up to 65536 state rows (batch x nheads x headdim)
+                                   where supported, else TC where supported, else SIMT */
     STREE_KERNEL_SIMT = 1,      /* CUDA-core fp32 kernel, every supported shape */
-    STREE_KERNEL_TC = 2         /* tcgen05 kernel; STREE_ERR_UNSUPPORTED if the shape is not */
+    STREE_KERNEL_TC = 2,        /* tcgen05 kernel; STREE_ERR_UNSUPPORTED if the shape is not */
+    STREE_KERNEL_SMALL = 3      /* small-batch CUDA-core kernel (dstate 128, headdim a multiple
+                                   of 32, n_nodes <= 64, a scan with y); else STREE_ERR_UNSUPPORTED */
 } stree_kernel;
 
 typedef struct stree_ctx stree_ctx;
@@ -109,6 +112,24 @@ stree_status stree_ctx_set_kernel(stree_ctx *ctx, stree_kernel kernel);
 /* Number of CUDA kernels this context has launched so far (host counter). */
 stree_status stree_ctx_launch_count(stree_ctx *ctx, int64_t *count);
 
+/* The kernel (SIMT, TC or SMALL) that ran the last scan call on this context;
+ * STREE_KERNEL_AUTO before the first one. */
+stree_status stree_ctx_last_kernel(stree_ctx *ctx, stree_kernel *kernel);
+
+/* Limit, in nanoseconds of device time, of every bounded wait inside the
+ * tensor-core kernel for later calls on this context (0, the default, means
+ * about 1 s).  A wait that runs out latches STREE_ERR_TIMEOUT; the CTA then does
+ * no further work, waits (bounded) for its own copies and MMAs in flight, frees
+ * its tensor memory and exits, and the context stays usable. */
+stree_status stree_ctx_set_wait_limit(stree_ctx *ctx, uint64_t ns);
+
+/* Test hook of that failure path: with fault = 1, later tensor-core scans on this
+ * context withhold one hand-off between two of the kernel's warp roles (the first
+ * tile's coefficients, on which no copy or MMA depends), so that a bounded wait
+ * runs out and the call reports STREE_ERR_TIMEOUT; 0 (the default) turns it off.
+ * Nothing faults or hangs the GPU.  Other values: STREE_ERR_INVALID_ARG. */
+stree_status stree_ctx_set_test_fault(stree_ctx *ctx, int fault);
+
 /*
  * Tree builder ("tree mask" of the packed sequence, STree summary "Approach"):
  * validates parent[] and builds the ancestor-or-self bitmask and depth of every
@@ -121,10 +142,11 @@ stree_status stree_build_tree(stree_ctx *ctx, const int32_t *parent, int n_nodes
 
 /*
  * Packed tree scan: y for every node of every sequence and head.  When parent is
- * not NULL the tree is (re)built first (as stree_build_tree); when it is NULL
- * the context's current tree is used and n_nodes / batch must match it.  The
- * input pointers are recorded for a later stree_commit (activation replay), so
- * x, dt, A, B and h0 must stay alive and unchanged until that commit.
+ * not NULL the tree is (re)built into the context by the same launch (with the
+ * checks and error reporting of stree_build_tree); when it is NULL the context's
+ * current tree is used and n_nodes / batch must match it.  The input pointers
+ * are recorded for a later stree_commit (activation replay), so x, dt, A, B and
+ * h0 must stay alive and unchanged until that commit.
  */
 stree_status stree_tree_scan(stree_ctx *ctx, const void *x, const void *dt, const float *A,
                              const void *B, const void *C, const float *D, const float *h0,
@@ -165,10 +187,15 @@ stree_status stree_tree_scan_commit(stree_ctx *ctx, const void *x, const void *d
  *
  * Scratch: the tree masks, depths and flags (and the CUDA-core kernel's C.B
  * pair scratch) live in one file-scope device array of 8 MiB that every GPU
- * loading the library keeps until the process exits.  Sizes whose scratch does
- * not fit return STREE_ERR_UNSUPPORTED before anything is launched.  The first
- * call on a device looks the array's device address up (cudaGetSymbolAddress);
- * make that first call before any stream capture.  Every call on a device
+ * loading the library keeps until the process exits.  With lazy module loading
+ * (the CUDA default) the array is placed on a device when the library's code is
+ * first loaded there, at the latest by the first call of this entry point on that
+ * device: a caller that will later run at its memory cap should make one call (a
+ * warm-up) before it reaches the cap, and before any stream capture, since that
+ * first call also looks the array's device address up (cudaGetSymbolAddress).  A
+ * call that finds a new CUDA context on the device (after cudaDeviceReset) looks
+ * the address up again.  Sizes whose scratch does not fit return
+ * STREE_ERR_UNSUPPORTED before anything is launched.  Every call on a device
  * shares the array, so calls that overlap on the GPU (other streams, other host
  * threads) race; serialise them.  The call never calls cudaMalloc or cudaFree.
  */

@@ -102,7 +102,7 @@ def test_binding_argtypes_match_header(lib_path):
         assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
         if name.startswith("stree_") and fn.argtypes and name not in (
                 "stree_status_string", "stree_ctx_create", "stree_ctx_destroy"):
-            args = [0 if t is ctypes.c_int else None for t in fn.argtypes]
+            args = [0 if t in (ctypes.c_int, ctypes.c_uint64, ctypes.c_float) else None for t in fn.argtypes]
             # NULL context / zero sizes: rejected on the host before any device work.
             assert fn(*args) in (1, 2), name
 

@@ -17,7 +17,7 @@ from gpu_util import TOL, assert_close, f64, i32, to_dev, upload_layer, upload_t
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = ["simt", "tc"]
+KERNELS = ["simt", "tc", "small"]
 
 
 @pytest.fixture(scope="module")
@@ -251,19 +251,21 @@ def test_invalid_tree_latches_error_and_skips(st, bad):
     assert torch.isfinite(y[0]).all() and not torch.all(y[0] == 7.0)
 
 
+@pytest.mark.parametrize("kernel", ["tc", "small"])
 @pytest.mark.parametrize("rebuild", [True, False], ids=["parent", "ctx_tree"])
 @pytest.mark.parametrize("bad", [[-1, 0, 0, 0, 1, 1, 2, 2, 3, 3, 4, 5, 6, 7, 15],
                                  [0, 0, 0, 0, 1, 1, 2, 2, 3, 3, 4, 5, 6, 7, 8],
                                  [-1, 0, 0, 0, 1, 1, 2, 2, 3, 3, 4, 5, 6, 13, 8]])
-def test_tc_invalid_tree_skips_only_that_sequence(st, rebuild, bad):
-    """Tensor-core kernel (bf16, dstate 128) with an invalid middle sequence: its masks
-    built in-kernel from parent[] (parent passed) or read from the context's tree
-    (built by an earlier call).  The builder reports the tree; the kernel writes
-    neither y nor h_new of that sequence and the others stay exact."""
+def test_invalid_tree_skips_only_that_sequence(st, kernel, rebuild, bad):
+    """Tensor-core and small-batch kernels (bf16, dstate 128) with an invalid middle
+    sequence: its masks built in-kernel from parent[] (parent passed; the kernel
+    reports the tree) or read from the context's tree (built and reported by an
+    earlier call).  The kernel writes neither y nor h_new of that sequence and the
+    others stay exact."""
     par = list(wl.M2_PARENT_15)
     w = wl.custom_workload([par, par, par], nheads=4, headdim=64, dstate=128, dtype="bf16", seed=5, h0_std=0.1)
     w.parent[1] = bad
-    ctx = _ctx(st, "tc")
+    ctx = _ctx(st, kernel)
     d, tr = upload_layer(w), upload_tree(w)
     y = torch.full_like(d["x"], 7.0)
     h_new = torch.full_like(d["h0"], 7.0)
@@ -327,3 +329,97 @@ def test_host_argument_checks(st):
     with pytest.raises(st.StreeError) as e:
         st.stree_build_tree(ctx, big)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("kernel", ["tc", "small"])
+@pytest.mark.parametrize("path,plen", [([1, 3, -1, -1], 2), ([0, 2, 3, -1], 3), ([0, 1, 3, 3], 5),
+                                       ([0, 1, 4, 9], 4), ([0, 0, -1, -1], 2), ([0, 1, 3, -1], -1)])
+def test_invalid_path_on_the_fused_kernels(st, kernel, path, plen):
+    """An invalid accepted path on the tensor-core and small-batch kernels: the
+    error is latched, h_new of that sequence stays untouched, y is still exact."""
+    par = [-1, 0, 0, 1, 1, 2]
+    w = wl.custom_workload([par, par], nheads=2, headdim=64, dstate=128, dtype="bf16", seed=9, h0_std=0.1,
+                           path=[[0, 1, 3, -1], path], path_len=[3, plen])
+    ctx = _ctx(st, kernel)
+    d, tr = upload_layer(w), upload_tree(w)
+    y = torch.empty_like(d["x"])
+    h_new = torch.full_like(d["h0"], 7.0)
+    st.stree_tree_scan_commit(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], tr["parent"],
+                              tr["path"], tr["path_len"], y, h_new)
+    status, info = st.stree_sync_check(ctx, raise_on_error=False)
+    assert status == 4 and info[1] == 1
+    assert torch.all(h_new[1] == 7.0)
+    f = w.f64(0)
+    assert_close(f64(y), oracle_tree_scan(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["h0"], w.parent),
+                 "bf16", "y")
+    h_ref = oracle_commit(f["x"][:1], f["dt"][:1], f["A"], f["B"][:1], f["h0"][:1], w.parent[:1], w.path[:1],
+                          w.path_len[:1])[0]
+    assert_close(f64(h_new[:1]), h_ref, "bf16", "h_new of the valid sequence")
+
+
+@pytest.mark.parametrize("kernel", ["tc", "small"])
+def test_fused_call_leaves_the_tree_in_the_context(st, kernel):
+    """With parent[] the fused kernels rebuild the tree themselves (no builder launch)
+    and leave it in the context: the path resolver and a later parent=NULL layer use it."""
+    w = wl.make_workload("hyb8b" if kernel == "small" else "serve64", batch=3, layers=2)
+    ctx = _ctx(st, kernel)
+    tr = upload_tree(w)
+    n0 = st.stree_ctx_launch_count(ctx)
+    outs = []
+    for layer in range(2):
+        d = upload_layer(w, layer)
+        y = torch.empty_like(d["x"])
+        h_new = torch.empty_like(d["h0"])
+        st.stree_tree_scan_commit(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"],
+                                  tr["parent"] if layer == 0 else None, tr["path"], tr["path_len"], y, h_new)
+        outs.append((y, h_new))
+    assert st.stree_ctx_launch_count(ctx) - n0 == 2                     # one kernel per layer
+    leaf = torch.zeros((w.batch,), dtype=torch.int32, device="cuda")
+    st.stree_resolve_path(ctx, tr["path"], tr["path_len"], leaf)
+    st.stree_sync_check(ctx)
+    expect_leaf = [w.path[i, w.path_len[i] - 1] if w.path_len[i] else -1 for i in range(w.batch)]
+    assert leaf.tolist() == expect_leaf
+    for layer, (y, h_new) in enumerate(outs):
+        yr, hr = _oracle(w, layer)
+        assert_close(f64(y), yr, w.dtype, f"layer {layer} y")
+        assert_close(f64(h_new), hr, w.dtype, f"layer {layer} h_new")
+
+
+@pytest.mark.parametrize("name,batch", [("tiny", None), ("m2_2p7b", None), ("serve64", 4), ("wide256", 2),
+                                        ("wide256_chain", 2)])
+def test_commit_alone_matches_oracle(st, name, batch):
+    """stree_commit (the streaming replay kernel) after a scan: every element of h_new,
+    including paths longer than one staging chunk (the chain) and an empty path."""
+    w = wl.make_workload(name, batch=batch, layers=1)
+    if w.batch > 1:
+        w.path_len[1] = 0
+        w.path[1] = -1
+    ctx = st.stree_ctx_create()
+    d, tr = upload_layer(w), upload_tree(w)
+    y = torch.empty_like(d["x"])
+    st.stree_tree_scan(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], tr["parent"], y)
+    h_new = torch.empty_like(d["h0"])
+    st.stree_commit(ctx, tr["path"], tr["path_len"], h_new)
+    st.stree_sync_check(ctx)
+    f = w.f64(0)
+    h_ref = oracle_commit(f["x"], f["dt"], f["A"], f["B"], f["h0"], w.parent, w.path, w.path_len, nthreads=8)[0]
+    assert_close(f64(h_new), h_ref, w.dtype, f"{name} h_new")
+    if w.batch > 1:
+        assert torch.equal(h_new[1], d["h0"][1])                         # empty path keeps h0 exactly
+    st.stree_commit(ctx, tr["path"], tr["path_len"], d["h0"])            # in place
+    st.stree_sync_check(ctx)
+    assert_close(f64(d["h0"]), h_ref, w.dtype, f"{name} h_new in place")
+
+
+def test_commit_alone_reports_a_bad_path(st):
+    w = wl.custom_workload([[-1, 0, 0, 1], [-1, 0, 0, 1]], nheads=2, headdim=8, dstate=8, seed=2,
+                           path=[[0, 1, 3, -1], [0, 2, 3, -1]], path_len=[3, 3])
+    ctx = st.stree_ctx_create()
+    d, tr = upload_layer(w), upload_tree(w)
+    st.stree_tree_scan(ctx, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], tr["parent"],
+                       torch.empty_like(d["x"]))
+    h_new = torch.full_like(d["h0"], 7.0)
+    st.stree_commit(ctx, tr["path"], tr["path_len"], h_new)
+    status, info = st.stree_sync_check(ctx, raise_on_error=False)
+    assert status == 4 and info[1] == 1 and info[2] == 1
+    assert torch.all(h_new[1] == 7.0) and not torch.all(h_new[0] == 7.0)

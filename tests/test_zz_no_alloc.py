@@ -4,15 +4,16 @@ stree_tree_scan_commit_noalloc serves callers that may not allocate device
 memory where they run the scan (a runtime that owns all device memory through
 its own pool, a process at its memory cap, a loop where an allocator call would
 synchronise).  It takes its scratch from the library's fixed device array, so
-its results must match stree_tree_scan_commit, which uses a context's workspace.
-Two calls in a row check that leftovers in the shared array never leak into the
-next result.  This file is collected last on purpose.
+its results must match stree_tree_scan_commit, which uses a context's workspace,
+and the fp64 oracle.  Two calls in a row check that leftovers in the shared
+array never leak into the next result.  This file is collected last on purpose.
 """
 import numpy as np
 import pytest
 import torch
 
 from hybrid_packed_tree_b200 import workloads as wl
+from oracle import oracle_commit, oracle_tree_scan
 
 from gpu_util import TOL, assert_close, f64, upload_layer, upload_tree
 
@@ -53,6 +54,29 @@ def test_noalloc_matches_context_entry_point_twice(st, name, batch):
         assert err.tolist() == [0, 0, 0, 0]
         assert_close(f64(y), f64(y_ref), w.dtype, f"{name} y")
         assert_close(f64(h_new), f64(h_ref), w.dtype, f"{name} h_new")
+    # And against the oracle, so that a layout fault of the scratch shared by
+    # both calls cannot pass unseen.
+    f = w.f64(0)
+    y_or = oracle_tree_scan(f["x"], f["dt"], f["A"], f["B"], f["C"], f["D"], f["h0"], w.parent, nthreads=8)
+    h_or = oracle_commit(f["x"], f["dt"], f["A"], f["B"], f["h0"], w.parent, w.path, w.path_len, nthreads=8)[0]
+    assert_close(f64(y), y_or, w.dtype, f"{name} y against the oracle")
+    assert_close(f64(h_new), h_or, w.dtype, f"{name} h_new against the oracle")
+
+
+def test_noalloc_batch_zero_is_a_no_op_like_the_context_call(st):
+    x = torch.empty((0, 5, 2, 8), device="cuda")
+    dt = torch.empty((0, 5, 2), device="cuda")
+    B = torch.empty((0, 5, 1, 8), device="cuda")
+    h0 = torch.empty((0, 2, 8, 8), device="cuda")
+    A = torch.ones(2, device="cuda")
+    parent = torch.empty((0, 5), dtype=torch.int32, device="cuda")
+    path = torch.empty((0, 0), dtype=torch.int32, device="cuda")        # maxlen 0
+    plen = torch.empty((0,), dtype=torch.int32, device="cuda")
+    ctx = st.stree_ctx_create()
+    st.stree_tree_scan_commit(ctx, x, dt, A, B, B, A, h0, parent, path, plen, torch.empty_like(x),
+                              torch.empty_like(h0))
+    st.stree_tree_scan_commit_noalloc(x, dt, A, B, B, A, h0, parent, path, plen, torch.empty_like(x),
+                                      torch.empty_like(h0))
 
 
 def test_noalloc_reports_a_bad_path_in_its_error_word(st):
