@@ -40,7 +40,7 @@ EXPORTS = (
     "stree_ctx_last_kernel", "stree_ctx_set_wait_limit", "stree_ctx_set_test_fault",
     "stree_build_tree",
     "stree_tree_scan", "stree_commit", "stree_tree_scan_commit", "stree_tree_scan_commit_noalloc",
-    "stree_resolve_path", "stree_unrolled_scan", "stree_accept_greedy",
+    "stree_resolve_path", "stree_unrolled_scan", "stree_accept_greedy", "stree_accept_sampling",
     "stree_sync_check", "stree_status_string", "stree_version",
 )
 
@@ -60,6 +60,8 @@ _lib.stree_tree_scan_commit_noalloc.argtypes = [_vp] * 8 + [_i] * 7 + [_vp, _vp,
 _lib.stree_resolve_path.argtypes = [_vp, _vp, _vp, _i, _vp, _vp]
 _lib.stree_unrolled_scan.argtypes = [_vp] * 9 + [_i] * 9 + [_vp, _vp, _vp, _vp]
 _lib.stree_accept_greedy.argtypes = [_vp, _i, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.stree_accept_sampling.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _i, _i, ctypes.c_float, _vp, _vp, _i, _vp,
+                                        _vp, _vp, _vp, _vp]
 _lib.stree_sync_check.argtypes = [_vp, _vp, _ip]
 _lib.stree_status_string.argtypes = [_i]
 _lib.stree_status_string.restype = ctypes.c_char_p
@@ -278,6 +280,29 @@ def stree_accept_greedy(logits, draft_tokens, parent, pred, accepted_path, path_
                                   _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
     _check(st, "stree_accept_greedy")
     return pred, accepted_path, path_len, bonus_token
+
+
+def stree_accept_sampling(target_logits, draft_logits, draft_tokens, parent, temperature, u_accept, u_bonus,
+                          accepted_path, path_len, bonus_token, err_out=None, stream=None):
+    """Stochastic tree verification by multi-step speculative sampling: (accepted_path,
+    path_len, bonus_token) from the target's and the draft's logits [b, T, V] (fp32 or
+    bf16, same dtype), the draft tokens [b, T] and the uniforms u_accept [b, T] and
+    u_bonus [b] (fp32)."""
+    batch, T, V = target_logits.shape
+    if draft_logits.shape != target_logits.shape or draft_logits.dtype != target_logits.dtype:
+        raise ValueError("draft_logits must match target_logits in shape and dtype")
+    st = _lib.stree_accept_sampling(_ptr(target_logits, "target_logits", (torch.float32, torch.bfloat16)),
+                                    _ptr(draft_logits, "draft_logits", (target_logits.dtype,)),
+                                    _io_dtype(target_logits), V, _ptr(draft_tokens, "draft_tokens", (torch.int32,)),
+                                    _ptr(parent, "parent", (torch.int32,)), T, batch, float(temperature),
+                                    _ptr(u_accept, "u_accept", (torch.float32,)),
+                                    _ptr(u_bonus, "u_bonus", (torch.float32,)), accepted_path.shape[1],
+                                    _ptr(accepted_path, "accepted_path", (torch.int32,)),
+                                    _ptr(path_len, "path_len", (torch.int32,)),
+                                    _ptr(bonus_token, "bonus_token", (torch.int32,)),
+                                    _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
+    _check(st, "stree_accept_sampling")
+    return accepted_path, path_len, bonus_token
 
 
 def stree_resolve_path(ctx: Ctx, path, path_len, leaf_out, stream=None):

@@ -188,6 +188,41 @@ def acceptance_inputs(parent: np.ndarray, vocab: int, seed: int = 7, dtype: str 
     return logits, tokens, planted
 
 
+def sampling_inputs(parent: np.ndarray, vocab: int, seed: int = 11, dtype: str = "bf16",
+                    draft_std: float = 3.0, target_noise: float = 0.5):
+    """Synthetic inputs for stochastic tree verification: draft logits ~ N(0,
+    draft_std), target logits = draft logits + N(0, target_noise) (a draft close to
+    the target), children's tokens distinct, each from the parent's four largest
+    draft logits with probability 0.7 and uniform over the vocabulary otherwise,
+    and the uniforms (u_accept [b,T], u_bonus [b], fp32 in [0, 1)).  Returns
+    (target, draft) logits [b,T,V] (fp32, or bf16 bits), tokens, u_accept, u_bonus."""
+    parent = np.asarray(parent)
+    rng = np.random.default_rng(seed)
+    b, T = parent.shape
+    draft = rng.normal(0.0, draft_std, size=(b, T, vocab)).astype(np.float32)
+    target = (draft + rng.normal(0.0, target_noise, size=(b, T, vocab))).astype(np.float32)
+    tokens = np.zeros((b, T), np.int32)
+    for s_ in range(b):
+        for u in range(T):
+            kids = np.nonzero(parent[s_] == u)[0]
+            if not len(kids):
+                continue
+            top = np.argsort(draft[s_, u])[-4:]
+            used = set()
+            for c in kids:
+                while True:
+                    t = int(rng.choice(top)) if rng.uniform() < 0.7 else int(rng.integers(vocab))
+                    if t not in used:
+                        break
+                used.add(t)
+                tokens[s_, c] = t
+    u_accept = rng.uniform(size=(b, T)).astype(np.float32)
+    u_bonus = rng.uniform(size=b).astype(np.float32)
+    if dtype == "bf16":
+        target, draft = bf16_bits(target), bf16_bits(draft)
+    return target, draft, tokens, u_accept, u_bonus
+
+
 # --------------------------------------------------------------------------- workloads
 
 

@@ -263,6 +263,44 @@ stree_status stree_accept_greedy(const void *logits, stree_dtype logit_dtype, in
                                  int32_t *bonus_token, int32_t *err_out, void *stream);
 
 /*
+ * Stochastic verification of the draft tree by multi-step speculative sampling
+ * (STree summary, "Builds on": SpecInfer and speculative sampling, the setting at
+ * temperature > 0; TreeSpark summary, "Guaranteeing Lossless Decoding": residual
+ * resampling).  At the current node u, with target distribution
+ * p = softmax(target_logits[u] / temperature) and draft distribution
+ * q = softmax(draft_logits[u] / temperature) (from which the tokens of u's
+ * children were drawn), the children are tried in increasing node order: child c
+ * with token t is accepted when u_accept[c] * q[t] < p[t], i.e. with probability
+ * min(1, p[t] / q[t]), and the walk continues from c; after each rejection p
+ * becomes max(p - q, 0) renormalised (unchanged when that is all zero).  When no
+ * child is accepted, u is a leaf or the path holds maxlen nodes, the bonus token
+ * is drawn from the current p by inverse CDF: the first token whose cumulative
+ * probability exceeds u_bonus times the total (the last token if none does).
+ *
+ *   target_logits, draft_logits [batch, n_nodes, vocab] fp32 or bf16 (logit_dtype), finite
+ *   draft_tokens  [batch, n_nodes] int32: the token of each node (root's unused), in [0, vocab)
+ *   parent        [batch, n_nodes] int32: the packed tree (as for the scan)
+ *   temperature   > 0
+ *   u_accept      [batch, n_nodes] fp32 in [0, 1): the uniform of each node, used when it is tried
+ *   u_bonus       [batch] fp32 in [0, 1): the uniform of the bonus draw
+ *   accepted_path [batch, maxlen] int32: receives the root-first accepted nodes, -1 after
+ *   path_len      [batch] int32: receives the number of accepted nodes (>= 1)
+ *   bonus_token   [batch] int32: receives the bonus token
+ *   err_out       device int32[4] error word of this call (cleared by the call), or NULL
+ *
+ * All arithmetic is fp32.  vocab up to 53248 (the current distribution is kept
+ * on chip); n_nodes up to 256.  An invalid tree latches STREE_ERR_BAD_TREE and a
+ * draft token outside [0, vocab) STREE_ERR_INVALID_ARG (position, token) for
+ * that sequence, which gets path_len 0, bonus -1 and a path of -1.  The caller
+ * owns every buffer; the call allocates nothing and runs on `stream`.
+ */
+stree_status stree_accept_sampling(const void *target_logits, const void *draft_logits, stree_dtype logit_dtype,
+                                   int vocab, const int32_t *draft_tokens, const int32_t *parent, int n_nodes,
+                                   int batch, float temperature, const float *u_accept, const float *u_bonus,
+                                   int maxlen, int32_t *accepted_path, int32_t *path_len, int32_t *bonus_token,
+                                   int32_t *err_out, void *stream);
+
+/*
  * Resolve accepted paths against the context's current tree: leaf_out[b] (device
  * int32 [batch]) receives the last node of a valid path, -1 for an empty path and
  * -2 for an invalid one (which also latches STREE_ERR_BAD_PATH).

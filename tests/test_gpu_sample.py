@@ -1,0 +1,131 @@
+"""Stochastic tree verification (stree_accept_sampling) against the oracle.
+
+The results are integers (path, length, bonus token), but floating point decides
+them: the kernel compares u * q[t] with p[t] and walks a CDF in fp32, the oracle
+in fp64.  Where a decision lies within rounding of its threshold the two may
+differ legitimately, so each case is first probed on the oracle alone: it is
+re-run with the logits and uniforms perturbed by a few fp32 ulps' worth of
+relative noise.  A sequence whose result survives every perturbation must match
+the oracle exactly; for the others (near-ties) the kernel's answer must be one
+of the oracle's answers under perturbation.  Each case also requires that most
+sequences are stable, so the exact comparison is never vacuous.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from hybrid_packed_tree_b200 import workloads as wl
+from oracle import oracle_accept_sampling
+
+from gpu_util import i32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def st():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from hybrid_packed_tree_b200 import stree
+    return stree
+
+
+def _logits(a, dtype):
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def _f64(a, dtype):
+    return wl.stored_to_f64(a, dtype)
+
+
+def _run(st, tl, dl, tokens, parent, temp, ua, ub, maxlen, dtype):
+    b, T = tokens.shape
+    path = torch.full((b, maxlen), -7, dtype=torch.int32, device="cuda")
+    plen = torch.full((b,), -7, dtype=torch.int32, device="cuda")
+    bonus = torch.full((b,), -7, dtype=torch.int32, device="cuda")
+    err = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    st.stree_accept_sampling(_logits(tl, dtype), _logits(dl, dtype), i32(tokens), i32(parent), temp,
+                             torch.from_numpy(np.ascontiguousarray(ua, np.float32)).cuda(),
+                             torch.from_numpy(np.ascontiguousarray(ub, np.float32)).cuda(), path, plen, bonus,
+                             err_out=err)
+    torch.cuda.synchronize()
+    return path.cpu().numpy(), plen.cpu().numpy(), bonus.cpu().numpy(), err.tolist()
+
+
+def test_sampling_golden_cases(st):
+    with open(os.path.join(os.path.dirname(__file__), "golden", "accept_sampling.json")) as f:
+        doc = json.load(f)
+    for c in doc["cases"]:
+        path, plen, bonus, err = _run(st, np.asarray(c["target_logits"], np.float32)[None],
+                                      np.asarray(c["draft_logits"], np.float32)[None],
+                                      np.asarray([c["tokens"]], np.int32), np.asarray([c["parent"]], np.int32),
+                                      doc["temperature"], np.asarray([c["u_accept"]]), np.asarray([c["u_bonus"]]),
+                                      c["maxlen"], "f32")
+        n = c["path_len"]
+        assert err == [0, 0, 0, 0], c["name"]
+        assert int(plen[0]) == n and path[0, :n].tolist() == c["path"] and (path[0, n:] == -1).all(), c["name"]
+        assert int(bonus[0]) == c["bonus"], c["name"]
+
+
+CASES = [
+    # (workload, batch, vocab, logits dtype, temperature, maxlen or None = n_nodes)
+    ("m2_2p7b", None, 50280, "bf16", 1.0, None),
+    ("serve64", 4, 50280, "bf16", 0.7, None),
+    ("serve64", 64, 4096, "f32", 1.0, None),
+    ("hyb8b", None, 1001, "f32", 1.3, 3),
+    ("wide256", 2, 777, "bf16", 1.0, None),
+    ("wide256_chain", 2, 333, "f32", 0.5, None),
+]
+
+
+@pytest.mark.parametrize("name,batch,vocab,dtype,temp,maxlen", CASES)
+def test_sampling_matches_oracle(st, name, batch, vocab, dtype, temp, maxlen):
+    w = wl.make_workload(name, batch=batch, layers=1)
+    maxlen = maxlen or w.n_nodes
+    tl, dl, tokens, ua, ub = wl.sampling_inputs(w.parent, vocab, seed=21, dtype=dtype)
+    t64, d64 = _f64(tl, dtype), _f64(dl, dtype)
+    ua64, ub64 = ua.astype(np.float64), ub.astype(np.float64)
+    ref = oracle_accept_sampling(t64, d64, tokens, w.parent, temp, ua64, ub64, maxlen)
+    rng = np.random.default_rng(5)
+    alts = []
+    for _ in range(4):
+        eps = 4e-6
+        alts.append(oracle_accept_sampling(t64 * (1 + eps * rng.standard_normal(t64.shape)),
+                                           d64 * (1 + eps * rng.standard_normal(d64.shape)), tokens, w.parent, temp,
+                                           ua64 * (1 + eps * rng.standard_normal(ua64.shape)),
+                                           ub64 * (1 + eps * rng.standard_normal(ub64.shape)), maxlen))
+    path, plen, bonus, err = _run(st, tl, dl, tokens, w.parent, temp, ua, ub, maxlen, dtype)
+    assert err == [0, 0, 0, 0]
+
+    def same(res, s):
+        p, n, bo = res
+        return int(n[s]) == int(plen[s]) and np.array_equal(p[s], path[s]) and int(bo[s]) == int(bonus[s])
+
+    stable = 0
+    for s in range(w.batch):
+        if all(int(a[1][s]) == int(ref[1][s]) and np.array_equal(a[0][s], ref[0][s]) and int(a[2][s]) == int(ref[2][s])
+               for a in alts):
+            stable += 1
+            assert same(ref, s), (name, s, path[s], plen[s], bonus[s], ref[0][s], ref[1][s], ref[2][s])
+        else:
+            assert same(ref, s) or any(same(a, s) for a in alts), (name, s)
+    assert stable >= max(1, int(0.8 * w.batch)), (name, stable, w.batch)
+    assert (plen >= 1).all() and (plen <= maxlen).all()
+    if w.batch >= 4:                     # the draft is close to the target: walks go past the root
+        assert plen.max() >= 2
+
+
+def test_sampling_reports_bad_trees_and_tokens(st):
+    parent = np.asarray([[-1, 0, 0, 1], [-1, 0, 3, 1], [-1, 0, 0, 1]], np.int32)
+    tl, dl, tokens, ua, ub = wl.sampling_inputs(np.asarray([[-1, 0, 0, 1]] * 3), 50, seed=2, dtype="f32")
+    tokens[2, 3] = 50                                        # outside the vocabulary
+    path, plen, bonus, err = _run(st, tl, dl, tokens, parent, 1.0, ua, ub, 4, "f32")
+    assert err[0] in (3, 1) and err[1] in (1, 2)
+    assert plen[1] == 0 and bonus[1] == -1 and (path[1] == -1).all()
+    assert plen[2] == 0 and bonus[2] == -1 and (path[2] == -1).all()
+    assert plen[0] >= 1
