@@ -13,6 +13,8 @@ load or call it, and the two share no code.
                multi-step speculative sampling; the accepted path and bonus token.
 * ``attention`` -- tree-masked attention of the hybrid model's Transformer layers
                over the packed tree (context plus each node's root path).
+* ``gdn``    -- the gated delta rule (linear-attention layers) over the packed tree:
+               the root-path walk, its commit, and a packed cross-check.
 """
 from .walk import (  # noqa: F401
     build_oracle,
@@ -23,3 +25,4 @@ from .walk import (  # noqa: F401
 )
 from .accept import oracle_accept_greedy, oracle_accept_sampling  # noqa: F401,E402
 from .attention import oracle_tree_attention  # noqa: F401,E402
+from .gdn import oracle_gdn_commit, oracle_gdn_tree  # noqa: F401,E402
