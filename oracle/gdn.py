@@ -42,6 +42,13 @@ def _path(parent_row, i):
     return out[::-1]
 
 
+def _step(S, kj, vj, a, be):
+    """One step of the rule: alpha S (I - beta k k^T) + beta v k^T, with the erase
+    applied as the rank-1 product S - beta (S k) k^T (the same matrix product,
+    without forming the d_k x d_k factor)."""
+    return a * (S - be * np.outer(S @ kj, kj)) + be * np.outer(vj, kj)
+
+
 def _f64(*arrays):
     return [np.asarray(a, np.float64) for a in arrays]
 
@@ -55,7 +62,6 @@ def oracle_gdn_tree(q, k, v, alpha, beta, S0, parent):
     Hv, dv = v.shape[2], v.shape[3]
     grp = Hv // Hk
     o = np.zeros((b, T, Hv, dv))
-    eye = np.eye(dk)
     for s in range(b):
         for i in range(T):
             path = _path(parent[s], i)
@@ -63,8 +69,7 @@ def oracle_gdn_tree(q, k, v, alpha, beta, S0, parent):
                 g = h // grp
                 S = S0[s, h].copy()
                 for j in path:
-                    kj = k[s, j, g]
-                    S = alpha[s, j, h] * S @ (eye - beta[s, j, h] * np.outer(kj, kj)) + beta[s, j, h] * np.outer(v[s, j, h], kj)
+                    S = _step(S, k[s, j, g], v[s, j, h], alpha[s, j, h], beta[s, j, h])
                 o[s, i, h] = S @ q[s, i, g]
     return o
 
@@ -78,7 +83,6 @@ def oracle_gdn_commit(k, v, alpha, beta, S0, parent, path, path_len):
     b, T, Hk, dk = k.shape
     Hv = v.shape[2]
     grp = Hv // Hk
-    eye = np.eye(dk)
     out = S0.copy()
     for s in range(b):
         n = int(path_len[s])
@@ -89,8 +93,7 @@ def oracle_gdn_commit(k, v, alpha, beta, S0, parent, path, path_len):
             g = h // grp
             S = S0[s, h].copy()
             for j in nodes:
-                kj = k[s, j, g]
-                S = alpha[s, j, h] * S @ (eye - beta[s, j, h] * np.outer(kj, kj)) + beta[s, j, h] * np.outer(v[s, j, h], kj)
+                S = _step(S, k[s, j, g], v[s, j, h], alpha[s, j, h], beta[s, j, h])
             out[s, h] = S
     return out
 

@@ -146,12 +146,12 @@ def test_packed_triangular_solve_equals_the_walk():
 def test_gdn_pins_catch_planted_mistakes():
     import oracle.gdn as gd
     src = open(gd.__file__).read()
-    step = "S = alpha[s, j, h] * S @ (eye - beta[s, j, h] * np.outer(kj, kj)) + beta[s, j, h] * np.outer(v[s, j, h], kj)"
-    assert src.count(step) == 2
+    step = "    return a * (S - be * np.outer(S @ kj, kj)) + be * np.outer(vj, kj)\n"
+    assert src.count(step) == 1
     mutants = {
-        "gate after the write": (step, "S = alpha[s, j, h] * (S @ (eye - beta[s, j, h] * np.outer(kj, kj)) + beta[s, j, h] * np.outer(v[s, j, h], kj))"),
-        "no beta on the write": (step, "S = alpha[s, j, h] * S @ (eye - beta[s, j, h] * np.outer(kj, kj)) + np.outer(v[s, j, h], kj)"),
-        "no erase (plain linear attention)": (step, "S = alpha[s, j, h] * S + beta[s, j, h] * np.outer(v[s, j, h], kj)"),
+        "gate after the write": (step, "    return a * (S - be * np.outer(S @ kj, kj) + be * np.outer(vj, kj))\n"),
+        "no beta on the write": (step, "    return a * (S - be * np.outer(S @ kj, kj)) + np.outer(vj, kj)\n"),
+        "no erase (plain linear attention)": (step, "    return a * S + be * np.outer(vj, kj)\n"),
         "heads round robin": ("                g = h // grp\n                S = S0[s, h].copy()\n                for j in path:",
                               "                g = h % Hk\n                S = S0[s, h].copy()\n                for j in path:"),
         "root skipped": ("    return out[::-1]\n", "    return out[::-1][1:]\n"),
