@@ -63,6 +63,8 @@ def parse():
                     help="skip the unrolled-tree baseline comparison (one layer per workload)")
     ap.add_argument("--no-accept", action="store_true",
                     help="skip the greedy tree-verification timing (argmax over the logits + walk)")
+    ap.add_argument("--no-gdn", action="store_true",
+                    help="skip the gated-delta-rule tree timing (linear-attention layers)")
     ap.add_argument("--vocab", type=int, default=50280,
                     help="vocabulary of the synthetic logits for the verification timing (Mamba2-2.7B's padded vocab)")
     return ap.parse_args()
@@ -339,6 +341,145 @@ def run_accept(name, vocab, local_rank, steps=20):
     return {"workload": name, "vocab": vocab, "logits_dtype": "bf16", "ms_per_call": ms, "bytes_per_call": nbytes,
             "achieved_gbs": gbs, "frac": gbs / hbm_gbs, "peak_source": f"{peak_kind} hbm_gbs",
             "timing": f"{steps} calls in one CUDA graph after an L2 flush, {nsets} distinct logits buffers"}
+
+
+def gdn_bytes(b, T, Hv, Hk, dk, dv, e, maxlen, nodes_on_paths):
+    """Bytes of one gated-delta-rule tree call with commit: S0 read and S_new
+    written (fp32), q, k, v, o, the gates, the tree and the paths."""
+    return (2 * b * Hv * dv * dk * 4 + 2 * b * T * Hk * dk * e + 2 * b * T * Hv * dv * e + 2 * b * T * Hv * 4
+            + b * T * 4 + b * maxlen * 4 + b * 4)
+
+
+def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16):
+    """The gated delta rule over a workload's trees (one linear-attention layer:
+    32 value heads, 16 query/key heads, d_k = d_v = 128, bf16 inputs, fp32 state),
+    fused with the commit of the workload's accepted paths; a CUDA graph of `steps`
+    calls over rotated buffers after an L2 flush."""
+    import torch
+
+    from hybrid_packed_tree_b200 import stree
+    from hybrid_packed_tree_b200 import workloads as wl
+
+    device = torch.device("cuda", local_rank)
+    w = wl.make_workload(name, layers=1)
+    g = wl.gdn_inputs(w.parent, w.path, w.path_len, heads_v=heads_v, heads_k=heads_k, dtype="bf16", seed=41)
+    b, T = w.parent.shape
+    nbytes = gdn_bytes(b, T, heads_v, heads_k, 128, 128, 2, w.maxlen, int(np.sum(w.path_len)))
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nsets = max(1, -(-3 * l2 // nbytes))
+    sets = []
+    for _ in range(nsets):
+        d = {k: dev_tensor(torch, getattr(g, k), "bf16", device) for k in ("q", "k", "v")}
+        d.update({k: dev_tensor(torch, getattr(g, k), "f32", device) for k in ("alpha", "beta", "S0")})
+        d.update({k: torch.from_numpy(np.ascontiguousarray(getattr(g, k))).to(device)
+                  for k in ("parent", "path", "path_len")})
+        d["o"] = torch.empty_like(d["v"])
+        d["S_new"] = torch.empty_like(d["S0"])
+        sets.append(d)
+    err = torch.zeros(4, dtype=torch.int32, device=device)
+
+    def call(i):
+        d = sets[i % nsets]
+        stree.stree_gdn_tree_scan_commit(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], d["parent"],
+                                         d["o"], d["path"], d["path_len"], d["S_new"], err_out=err,
+                                         stream=torch.cuda.current_stream(device))
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize(device)
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for i in range(steps):
+            call(i)
+    gr.replay()
+    flush = torch.empty(int(3 * l2) // 4 + 1, dtype=torch.float32, device=device)
+    flush.zero_()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    gr.replay()
+    t1.record()
+    torch.cuda.synchronize(device)
+    if int(err[0]) != 0:
+        raise RuntimeError(f"device error in the gated-delta-rule step: {err.tolist()}")
+    ms = t0.elapsed_time(t1) / steps
+    del gr
+    hbm_gbs, peak_kind = peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"{name} trees, gated delta rule ({heads_v} value / {heads_k} key heads, d_k = d_v = 128)",
+            "batch": b, "n_nodes": T, "ms_per_call": ms, "nodes_per_s": b * T / (ms / 1e3),
+            "bytes_per_call": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs,
+            "peak_source": f"{peak_kind} hbm_gbs", "kernel": "gdn_tree_kernel",
+            "timing": f"{steps} calls in one CUDA graph after an L2 flush, {nsets} rotated buffer sets"}
+
+
+def run_sampling(name, vocab, local_rank, steps=20, temperature=1.0):
+    """Stochastic tree verification (stree_accept_sampling) on synthetic target and
+    draft logits [b, T, vocab] (bf16) of a workload's trees, timed as a CUDA graph of
+    `steps` calls after an L2 flush.  Its algorithmic bytes are the logits rows of
+    the nodes the walks visit (target and draft; the residual passes re-read a draft
+    row from L2), counted from the returned paths."""
+    import torch
+
+    from hybrid_packed_tree_b200 import stree
+    from hybrid_packed_tree_b200 import workloads as wl
+
+    device = torch.device("cuda", local_rank)
+    w = wl.make_workload(name, layers=1)
+    b, T = w.parent.shape
+    tl, dl, tokens, ua, ub = wl.sampling_inputs(w.parent, vocab, seed=21, dtype="bf16")
+    t_logits = [dev_tensor(torch, tl, "bf16", device)]
+    d_logits = [dev_tensor(torch, dl, "bf16", device)]
+    tok = torch.from_numpy(tokens).to(device)
+    par = torch.from_numpy(w.parent).to(device)
+    uat = torch.from_numpy(ua).to(device)
+    ubt = torch.from_numpy(ub).to(device)
+    path = torch.empty((b, T), dtype=torch.int32, device=device)
+    plen = torch.empty((b,), dtype=torch.int32, device=device)
+    bonus = torch.empty((b,), dtype=torch.int32, device=device)
+    err = torch.zeros(4, dtype=torch.int32, device=device)
+
+    def call(i):
+        stree.stree_accept_sampling(t_logits[i % len(t_logits)], d_logits[i % len(d_logits)], tok, par, temperature,
+                                    uat, ubt, path, plen, bonus, err_out=err, stream=torch.cuda.current_stream(device))
+
+    call(0)
+    torch.cuda.synchronize(device)
+    # Copies of the logits (same values, so the same walks) rotated so that the
+    # rows a call visits are not left in L2 by the calls before it.
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    visited = int(plen.sum().item())
+    nsets = max(1, min(steps, -(-3 * l2 // max(1, 2 * visited * vocab * 2))))
+    while len(t_logits) < nsets:
+        t_logits.append(t_logits[0].clone())
+        d_logits.append(d_logits[0].clone())
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            call(i)
+    g.replay()
+    flush = torch.empty(int(3 * l2) // 4 + 1, dtype=torch.float32, device=device)
+    flush.zero_()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    g.replay()
+    t1.record()
+    torch.cuda.synchronize(device)
+    if int(err[0]) != 0:
+        raise RuntimeError(f"device error in the sampling verification: {err.tolist()}")
+    ms = t0.elapsed_time(t1) / steps
+    del g
+    nbytes = 2 * visited * vocab * 2
+    hbm_gbs, peak_kind = peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": name, "vocab": vocab, "logits_dtype": "bf16", "temperature": temperature,
+            "ms_per_call": ms, "accepted_nodes": visited, "bytes_per_call": nbytes, "achieved_gbs": gbs,
+            "frac": gbs / hbm_gbs, "peak_source": f"{peak_kind} hbm_gbs",
+            "timing": f"{steps} calls in one CUDA graph after an L2 flush, {nsets} rotated copies of the logits"}
 
 
 def unrolled_summary(o, u):
@@ -733,10 +874,16 @@ def main():
                 out["other_workloads"][name]["unrolled_baseline"] = unrolled_summary(o2, run_unrolled(name, local_rank))
             if not args.no_accept and rank == 0 and name in SIDE_WORKLOADS:
                 out["other_workloads"][name]["accept_greedy"] = run_accept(name, args.vocab, local_rank)
+                out["other_workloads"][name]["accept_sampling"] = run_sampling(name, args.vocab, local_rank)
+            if not args.no_gdn and rank == 0 and name in SIDE_WORKLOADS:
+                out["other_workloads"][name]["gdn_tree"] = run_gdn(name, local_rank)
     if rank == 0 and not args.no_unrolled:
         out["unrolled_baseline"] = unrolled_summary(out, run_unrolled(args.config, local_rank))
     if rank == 0 and not args.no_accept:
         out["accept_greedy"] = run_accept(args.config, args.vocab, local_rank)
+        out["accept_sampling"] = run_sampling(args.config, args.vocab, local_rank)
+    if rank == 0 and not args.no_gdn:
+        out["gdn_tree"] = run_gdn(args.config, local_rank)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_seconds)
     if rank == 0:

@@ -14,15 +14,16 @@
 // Design.  The op streams the state (read h0, write h_new: 2 x 4 bytes per
 // element) and adds at most a path's worth of rank-1 terms, so it is HBM-bound.
 // One CTA per (sequence, head, slab of R = 8192 / dstate rows): the slab is
-// R x dstate contiguous fp32 (32 KB), eight 16-byte loads per thread issued at
-// entry, before the path is known, so the state is in flight during the two
-// dependent rounds of small loads (path; then dt, x and B at the path nodes).
-// The path's B rows and the per-row coefficients w_q x_q are staged in shared
-// memory sixteen path positions at a time.  Several CTAs per SM overlap one
-// another's round trips.
+// R x dstate contiguous fp32 (32 KB).  At entry one bulk request prefetches the
+// slab into L2 while the threads read the path; the second round (the checks of
+// every path position, dt, and the path's B rows and x values staged in shared
+// memory, sixteen positions at a time) is issued before the slab's register
+// loads, so the small dependent loads never queue behind the slab.  Several CTAs
+// per SM overlap one another's round trips.
 #include <climits>
 
 #include "stree_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace stree {
 namespace {
@@ -44,13 +45,33 @@ struct CommitParams {
     stree_dtype dtype;
 };
 
-__global__ void __launch_bounds__(kCThreads) commit_kernel(const CommitParams p)
+// Stages B rows and x values (of the slab's rows) of path positions q0 .. q0 + nq - 1;
+// node ids are clamped into range (an invalid path's values are never used).
+__device__ __forceinline__ void stage_path_rows(const CommitParams &p, float *Bq, float *cfq, const int32_t *pn,
+                                                int q0, int nq, int b, int h, int g, int p0, int rows)
+{
+    const int T = p.T, N = p.N;
+    const size_t xrow = (size_t)p.H * p.P;
+    for (int e = threadIdx.x; e < nq * N; e += kCThreads) {
+        const int qq = e / N, n = e - qq * N;
+        const int j = min(max(pn[q0 + qq], 0), T - 1);
+        Bq[qq * N + n] = load_as_float(p.B, (((size_t)b * T + j) * p.G + g) * N + n, p.dtype);
+    }
+    for (int e = threadIdx.x; e < nq * rows; e += kCThreads) {
+        const int qq = e / rows, r = e - qq * rows;
+        const int j = min(max(pn[q0 + qq], 0), T - 1);
+        cfq[qq * rows + r] = load_as_float(p.x, ((size_t)b * T + j) * xrow + (size_t)h * p.P + p0 + r, p.dtype);
+    }
+}
+
+__global__ void __launch_bounds__(kCThreads, 4) commit_kernel(const CommitParams p)
 {
     __shared__ __align__(16) float Bq[kQChunk * kMaxDim];   // staged path rows of B
-    __shared__ float cfq[kQChunk * kMaxDim];                // w_q x_q per slab row
+    __shared__ float cfq[kQChunk * kMaxDim];                // x_q per slab row
     __shared__ int32_t pn[kMaxNodes];
     __shared__ float dq[kMaxNodes], wq[kMaxNodes];
-    __shared__ int32_t s_badq;
+    __shared__ int32_t s_badq, s_ok, s_len;
+    __shared__ float s_A;
 
     const int tid = threadIdx.x;
     const int T = p.T, H = p.H, P = p.P, N = p.N, G = p.G, W = p.tree.W;
@@ -62,42 +83,71 @@ __global__ void __launch_bounds__(kCThreads) commit_kernel(const CommitParams p)
     const bool leader = h == 0 && chunk == 0;
     const int n4 = N / 4, nf = rows * n4;
 
-    // The state slab first: it does not depend on the path.
-    const float4 *src = reinterpret_cast<const float4 *>(p.h0 + (((size_t)b * H + h) * P + p0) * N);
-    float4 hv[kCVec];
-#pragma unroll
-    for (int k = 0; k < kCVec; ++k) {
-        const int f = tid + k * kCThreads;
-        hv[k] = f < nf ? __ldcs(src + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+    // Round one: the slab is prefetched into L2 by one bulk request (it does not
+    // depend on the path), and the path, its length and the tree flag are read.
+    const int plim = min(p.maxlen, T);
+    const float *slab = p.h0 + (((size_t)b * H + h) * P + p0) * N;
+    if (tid == 0) ptx::prefetch_l2(slab, (uint32_t)nf * 16u);
+    int pv = 0, okv = 0, lenv = 0;
+    float Av = 0.f;
+    if (tid < plim) pv = p.path[(size_t)b * p.maxlen + tid];
+    if (tid == 0) {
+        okv = p.tree.ok[b];
+        lenv = p.path_len[b];
+        Av = p.A[h];
     }
-    if (!p.tree.ok[b]) return;                     // invalid tree: h_new untouched
-    const int len = p.path_len[b];
+    if (tid < plim) pn[tid] = pv;
+    if (tid == 0) {
+        s_ok = okv;
+        s_len = lenv;
+        s_A = Av;
+        s_badq = INT_MAX;
+    }
+    __syncthreads();
+    const int len = s_len;
+    if (!s_ok) return;                             // invalid tree: h_new untouched
     if (len < 0 || len > p.maxlen || len > T) {
         if (leader && tid == 0) latch_error(p.err, STREE_ERR_BAD_PATH, b, -1, len);
         return;
     }
-    if (tid < len) pn[tid] = p.path[(size_t)b * p.maxlen + tid];
-    if (tid == 0) s_badq = INT_MAX;
-    __syncthreads();
 
-    // Position q must hold the depth-q ancestor of the last node.
+    // Round two, all at once: the checks of every path position (depth, the
+    // leaf's ancestor bit), dt at the path's nodes, and the first chunk's B rows
+    // and x values (node ids clamped into range; an invalid path discards them).
+    const int leaf = len > 0 ? pn[len - 1] : 0;
+    const bool leaf_ok = leaf >= 0 && leaf < T;
     int bad = 0;
     for (int q = tid; q < len; q += kCThreads) {
-        const int leaf = pn[len - 1], j = pn[q];
-        const bool good = leaf >= 0 && leaf < T && j >= 0 && j < T &&
-                          ((p.tree.anc[((size_t)b * T + leaf) * W + (j >> 5)] >> (j & 31)) & 1u) &&
+        const int j = pn[q];
+        const bool in = leaf_ok && j >= 0 && j < T;
+        const bool good = in && ((p.tree.anc[((size_t)b * T + leaf) * W + (j >> 5)] >> (j & 31)) & 1u) &&
                           p.tree.depth[(size_t)b * T + j] == q;
         if (!good) {
             bad = 1;
             atomicMin(&s_badq, q);
         }
-        dq[q] = good ? load_as_float(p.dt, ((size_t)b * T + j) * H + h, p.dtype) : 0.f;
+        dq[q] = in ? load_as_float(p.dt, ((size_t)b * T + j) * H + h, p.dtype) : 0.f;
+    }
+    stage_path_rows(p, Bq, cfq, pn, 0, min(kQChunk, len), b, h, g, p0, rows);
+    // The slab into registers (from L2 by now), issued after the small loads so
+    // that they are not queued behind it.
+    const float4 *src = reinterpret_cast<const float4 *>(slab);
+    float4 hv[kCVec];
+#pragma unroll
+    for (int k = 0; k < kCVec; ++k) {
+        const int f = tid + k * kCThreads;
+        hv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (f < nf)
+            asm volatile("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(hv[k].x), "=f"(hv[k].y), "=f"(hv[k].z), "=f"(hv[k].w)
+                         : "l"(src + f)
+                         : "memory");
     }
     if (__syncthreads_or(bad)) {
         if (leader && tid == 0) latch_error(p.err, STREE_ERR_BAD_PATH, b, s_badq, pn[s_badq]);
         return;
     }
-    const float Ah = __ldg(p.A + h);
+    const float Ah = s_A;
     if (tid == 0) {
         // L along the path (a prefix sum), then the replay weights.
         float s = 0.f;
@@ -115,18 +165,11 @@ __global__ void __launch_bounds__(kCThreads) commit_kernel(const CommitParams p)
     float4 acc[kCVec];
 #pragma unroll
     for (int k = 0; k < kCVec; ++k) acc[k] = make_float4(al * hv[k].x, al * hv[k].y, al * hv[k].z, al * hv[k].w);
-    const size_t xrow = (size_t)H * P;
     for (int q0 = 0; q0 < len; q0 += kQChunk) {
         const int nq = min(kQChunk, len - q0);
-        __syncthreads();
-        for (int e = tid; e < nq * N; e += kCThreads) {
-            const int qq = e / N, n = e - qq * N;
-            Bq[qq * N + n] = load_as_float(p.B, (((size_t)b * T + pn[q0 + qq]) * G + g) * N + n, p.dtype);
-        }
-        for (int e = tid; e < nq * rows; e += kCThreads) {
-            const int qq = e / rows, r = e - qq * rows;
-            const size_t xi = ((size_t)b * T + pn[q0 + qq]) * xrow + (size_t)h * P + p0 + r;
-            cfq[qq * rows + r] = wq[q0 + qq] * load_as_float(p.x, xi, p.dtype);
+        if (q0 > 0) {
+            __syncthreads();
+            stage_path_rows(p, Bq, cfq, pn, q0, nq, b, h, g, p0, rows);
         }
         __syncthreads();
 #pragma unroll
@@ -135,7 +178,7 @@ __global__ void __launch_bounds__(kCThreads) commit_kernel(const CommitParams p)
             if (f < nf) {
                 const int r = f / n4, c = f - r * n4;
                 for (int qq = 0; qq < nq; ++qq) {
-                    const float cf = cfq[qq * rows + r];
+                    const float cf = wq[q0 + qq] * cfq[qq * rows + r];
                     const float4 bv = *reinterpret_cast<const float4 *>(Bq + qq * N + 4 * c);
                     acc[k].x = fmaf(cf, bv.x, acc[k].x);
                     acc[k].y = fmaf(cf, bv.y, acc[k].y);

@@ -164,7 +164,7 @@ namespace stree {
 // small-batch kernel when both it and the tensor-core kernel support the shape:
 // below it a launch is bound by latency, which the small kernel's short chain
 // serves better than the tensor-core pipeline.
-constexpr long long kSmallRows = 65536;
+constexpr long long kSmallRows = 16384;
 
 bool select_path(stree_kernel sel, const ScanArgs &a, ScanPath *out)
 {

@@ -223,6 +223,72 @@ def sampling_inputs(parent: np.ndarray, vocab: int, seed: int = 11, dtype: str =
     return target, draft, tokens, u_accept, u_bonus
 
 
+@dataclass
+class GdnInputs:
+    """One gated-delta-rule layer over packed trees (bf16 q/k/v, fp32 gates and state)."""
+    q: np.ndarray          # [b, T, Hk, dk]  bf16 bits (or fp32)
+    k: np.ndarray          # [b, T, Hk, dk]  unit rows before rounding
+    v: np.ndarray          # [b, T, Hv, dv]
+    alpha: np.ndarray      # [b, T, Hv] fp32 in (0, 1]
+    beta: np.ndarray       # [b, T, Hv] fp32 in (0, 1)
+    S0: np.ndarray         # [b, Hv, dv, dk] fp32
+    parent: np.ndarray
+    path: np.ndarray
+    path_len: np.ndarray
+    dtype: str
+
+    def f64(self):
+        return {"q": stored_to_f64(self.q, self.dtype), "k": stored_to_f64(self.k, self.dtype),
+                "v": stored_to_f64(self.v, self.dtype), "alpha": self.alpha.astype(np.float64),
+                "beta": self.beta.astype(np.float64), "S0": self.S0.astype(np.float64)}
+
+
+def gdn_inputs(parent: np.ndarray, path: np.ndarray, path_len: np.ndarray, *, heads_v: int = 32,
+               heads_k: int = 16, dk: int = 128, dv: int = 128, seed: int = 31, dtype: str = "bf16",
+               s0_std: float = 0.1) -> GdnInputs:
+    """Seeded inputs of a gated-delta-rule layer on the given trees: q, k unit
+    vectors (Gaussian directions), v ~ N(0, 1), alpha = exp(-U(0.01, 0.3)),
+    beta = 1 / (1 + exp(-N(0, 1))), S0 ~ N(0, s0_std)."""
+    parent = np.asarray(parent, np.int32)
+    rng = np.random.default_rng(seed)
+    b, T = parent.shape
+
+    def unit(shape):
+        a = rng.normal(size=shape)
+        return a / np.linalg.norm(a, axis=-1, keepdims=True)
+
+    q = _round(unit((b, T, heads_k, dk)), dtype)
+    k = _round(unit((b, T, heads_k, dk)), dtype)
+    v = _round(rng.normal(size=(b, T, heads_v, dv)), dtype)
+    alpha = np.exp(-rng.uniform(0.01, 0.3, size=(b, T, heads_v))).astype(np.float32)
+    beta = (1.0 / (1.0 + np.exp(-rng.normal(size=(b, T, heads_v))))).astype(np.float32)
+    S0 = rng.normal(0.0, s0_std, size=(b, heads_v, dv, dk)).astype(np.float32)
+    return GdnInputs(q=q, k=k, v=v, alpha=alpha, beta=beta, S0=S0, parent=parent,
+                     path=np.asarray(path, np.int32), path_len=np.asarray(path_len, np.int32), dtype=dtype)
+
+
+def attention_inputs(parent: np.ndarray, ctx_cap: int, ctx_len, *, heads_q: int = 32, heads_kv: int = 8,
+                     head_dim: int = 128, seed: int = 51, stale=np.nan):
+    """Seeded inputs of a tree-masked attention layer (bf16 bits): q [b, T, Hq, d],
+    the context cache k_ctx, v_ctx [b, ctx_cap, Hkv, d] whose positions past each
+    sequence's ctx_len hold `stale` (they must never be read), and the tree's own
+    k_tree, v_tree [b, T, Hkv, d]; all valid values ~ N(0, 1)."""
+    parent = np.asarray(parent, np.int32)
+    rng = np.random.default_rng(seed)
+    b, T = parent.shape
+    ctx_len = np.asarray(ctx_len, np.int32).reshape(b)
+    q = bf16_bits(rng.normal(size=(b, T, heads_q, head_dim)).astype(np.float32))
+    kc = rng.normal(size=(b, ctx_cap, heads_kv, head_dim)).astype(np.float32)
+    vc = rng.normal(size=(b, ctx_cap, heads_kv, head_dim)).astype(np.float32)
+    for s_ in range(b):
+        kc[s_, ctx_len[s_]:] = stale
+        vc[s_, ctx_len[s_]:] = stale
+    kt = bf16_bits(rng.normal(size=(b, T, heads_kv, head_dim)).astype(np.float32))
+    vt = bf16_bits(rng.normal(size=(b, T, heads_kv, head_dim)).astype(np.float32))
+    return {"q": q, "k_ctx": bf16_bits(kc), "v_ctx": bf16_bits(vc), "k_tree": kt, "v_tree": vt,
+            "ctx_len": ctx_len, "parent": parent, "scale": 1.0 / np.sqrt(head_dim)}
+
+
 # --------------------------------------------------------------------------- workloads
 
 
