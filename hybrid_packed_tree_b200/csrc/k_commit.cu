@@ -12,14 +12,19 @@
 // so both give the same fp32 L).
 //
 // Design.  The op streams the state (read h0, write h_new: 2 x 4 bytes per
-// element) and adds at most a path's worth of rank-1 terms, so it is HBM-bound.
-// One CTA per (sequence, head, slab of R = 8192 / dstate rows): the slab is
-// R x dstate contiguous fp32 (32 KB).  At entry one bulk request prefetches the
-// slab into L2 while the threads read the path; the second round (the checks of
-// every path position, dt, and the path's B rows and x values staged in shared
-// memory, sixteen positions at a time) is issued before the slab's register
-// loads, so the small dependent loads never queue behind the slab.  Several CTAs
-// per SM overlap one another's round trips.
+// element) and adds at most a path's worth of rank-1 terms, so it is HBM-bound;
+// what must not happen is a chain of small dependent reads in front of every
+// slab.  Two launches:
+//   * commit_prep_kernel (one CTA per sequence): checks the path against the
+//     tree, and writes the path's nodes, its length (-1 when invalid) and for
+//     every head the weights w_q = exp(L_leaf - L_q) dt_q and exp(L_leaf) into a
+//     small workspace;
+//   * commit_stream_kernel (one CTA per (sequence, head, slab of R = 8192 /
+//     dstate rows), a programmatic dependent of the first): issues its 32 KB of
+//     h0 at entry -- h0 is not written by the prep launch -- then waits for the
+//     prep, reads the path and weights (L2), stages the path's B rows and x
+//     values in shared memory sixteen positions at a time, and writes h_new.
+// The first stream CTAs' state loads run while the prep launch works.
 #include <climits>
 
 #include "stree_internal.cuh"
@@ -38,15 +43,82 @@ struct CommitParams {
     const float *A, *h0;
     TreeView tree;
     const int32_t *path, *path_len;
-    int maxlen;
+    int maxlen, Lc;                          // Lc = min(maxlen, T): path slots in the workspace
     float *h_new;
     int32_t *err;
+    CommitWork ws;
     int T, H, P, N, G, R, chunks;
     stree_dtype dtype;
 };
 
-// Stages B rows and x values (of the slab's rows) of path positions q0 .. q0 + nq - 1;
-// node ids are clamped into range (an invalid path's values are never used).
+// One CTA per sequence: the path's check, nodes and length; per head the weights.
+__global__ void __launch_bounds__(kCThreads) commit_prep_kernel(const CommitParams p)
+{
+    __shared__ int32_t pn[kMaxNodes];
+    __shared__ int32_t s_badq, s_len;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int T = p.T, H = p.H, W = p.tree.W;
+    const int plim = min(p.maxlen, T);
+    if (tid < plim) pn[tid] = p.path[(size_t)b * p.maxlen + tid];
+    if (tid == 0) {
+        s_badq = INT_MAX;
+        const int len = p.path_len[b];
+        const bool ok = p.tree.ok[b] != 0;
+        s_len = !ok ? -1 : (len < 0 || len > p.maxlen || len > T) ? -2 : len;
+    }
+    __syncthreads();
+    const int len = s_len;
+    if (len == -2) {
+        if (tid == 0) {
+            latch_error(p.err, STREE_ERR_BAD_PATH, b, -1, p.path_len[b]);
+            p.ws.len[b] = -1;
+        }
+        return;
+    }
+    if (len < 0) {                                 // invalid tree: h_new untouched
+        if (tid == 0) p.ws.len[b] = -1;
+        return;
+    }
+    // Position q must hold the depth-q ancestor of the last node.
+    int bad = 0;
+    if (tid < len) {
+        const int leaf = pn[len - 1], j = pn[tid];
+        const bool good = leaf >= 0 && leaf < T && j >= 0 && j < T &&
+                          ((p.tree.anc[((size_t)b * T + leaf) * W + (j >> 5)] >> (j & 31)) & 1u) &&
+                          p.tree.depth[(size_t)b * T + j] == tid;
+        if (!good) {
+            bad = 1;
+            atomicMin(&s_badq, tid);
+        }
+    }
+    if (__syncthreads_or(bad)) {
+        if (tid == 0) {
+            latch_error(p.err, STREE_ERR_BAD_PATH, b, s_badq, pn[s_badq]);
+            p.ws.len[b] = -1;
+        }
+        return;
+    }
+    if (tid < len) p.ws.pn[(size_t)b * p.Lc + tid] = pn[tid];
+    if (tid == 0) p.ws.len[b] = len;
+    // Per head: L along the path (a prefix sum of dt in path order), then the weights.
+    for (int h = tid; h < H; h += kCThreads) {
+        const float Ah = p.A[h];
+        float s = 0.f;
+        for (int q = 0; q < len; ++q) s += load_as_float(p.dt, ((size_t)b * T + pn[q]) * H + h, p.dtype);
+        const float Lleaf = Ah * s;
+        float pre = 0.f;
+        float *wh = p.ws.w + ((size_t)b * H + h) * p.Lc;
+        for (int q = 0; q < len; ++q) {
+            const float d = load_as_float(p.dt, ((size_t)b * T + pn[q]) * H + h, p.dtype);
+            pre += d;
+            wh[q] = expf(Lleaf - Ah * pre) * d;
+        }
+        p.ws.alpha[(size_t)b * H + h] = len > 0 ? expf(Lleaf) : 1.f;
+    }
+}
+
+// Stages B rows and x values (of the slab's rows) of path positions q0 .. q0 + nq - 1.
 __device__ __forceinline__ void stage_path_rows(const CommitParams &p, float *Bq, float *cfq, const int32_t *pn,
                                                 int q0, int nq, int b, int h, int g, int p0, int rows)
 {
@@ -54,84 +126,34 @@ __device__ __forceinline__ void stage_path_rows(const CommitParams &p, float *Bq
     const size_t xrow = (size_t)p.H * p.P;
     for (int e = threadIdx.x; e < nq * N; e += kCThreads) {
         const int qq = e / N, n = e - qq * N;
-        const int j = min(max(pn[q0 + qq], 0), T - 1);
-        Bq[qq * N + n] = load_as_float(p.B, (((size_t)b * T + j) * p.G + g) * N + n, p.dtype);
+        Bq[qq * N + n] = load_as_float(p.B, (((size_t)b * T + pn[q0 + qq]) * p.G + g) * N + n, p.dtype);
     }
     for (int e = threadIdx.x; e < nq * rows; e += kCThreads) {
         const int qq = e / rows, r = e - qq * rows;
-        const int j = min(max(pn[q0 + qq], 0), T - 1);
-        cfq[qq * rows + r] = load_as_float(p.x, ((size_t)b * T + j) * xrow + (size_t)h * p.P + p0 + r, p.dtype);
+        cfq[qq * rows + r] = load_as_float(p.x, ((size_t)b * T + pn[q0 + qq]) * xrow + (size_t)h * p.P + p0 + r, p.dtype);
     }
 }
 
-__global__ void __launch_bounds__(kCThreads, 4) commit_kernel(const CommitParams p)
+__global__ void __launch_bounds__(kCThreads, 4) commit_stream_kernel(const CommitParams p)
 {
     __shared__ __align__(16) float Bq[kQChunk * kMaxDim];   // staged path rows of B
     __shared__ float cfq[kQChunk * kMaxDim];                // x_q per slab row
     __shared__ int32_t pn[kMaxNodes];
-    __shared__ float dq[kMaxNodes], wq[kMaxNodes];
-    __shared__ int32_t s_badq, s_ok, s_len;
-    __shared__ float s_A;
+    __shared__ float wq[kMaxNodes];
+    __shared__ int32_t s_len;
+    __shared__ float s_alpha;
 
     const int tid = threadIdx.x;
-    const int T = p.T, H = p.H, P = p.P, N = p.N, G = p.G, W = p.tree.W;
+    const int H = p.H, P = p.P, N = p.N, G = p.G;
     const int chunk = blockIdx.x % p.chunks;
     const int h = (blockIdx.x / p.chunks) % H;
     const int b = blockIdx.x / (p.chunks * H);
     const int g = h / (H / G);
     const int p0 = chunk * p.R, rows = min(p.R, P - p0);
-    const bool leader = h == 0 && chunk == 0;
     const int n4 = N / 4, nf = rows * n4;
 
-    // Round one: the slab is prefetched into L2 by one bulk request (it does not
-    // depend on the path), and the path, its length and the tree flag are read.
-    const int plim = min(p.maxlen, T);
-    const float *slab = p.h0 + (((size_t)b * H + h) * P + p0) * N;
-    if (tid == 0) ptx::prefetch_l2(slab, (uint32_t)nf * 16u);
-    int pv = 0, okv = 0, lenv = 0;
-    float Av = 0.f;
-    if (tid < plim) pv = p.path[(size_t)b * p.maxlen + tid];
-    if (tid == 0) {
-        okv = p.tree.ok[b];
-        lenv = p.path_len[b];
-        Av = p.A[h];
-    }
-    if (tid < plim) pn[tid] = pv;
-    if (tid == 0) {
-        s_ok = okv;
-        s_len = lenv;
-        s_A = Av;
-        s_badq = INT_MAX;
-    }
-    __syncthreads();
-    const int len = s_len;
-    if (!s_ok) return;                             // invalid tree: h_new untouched
-    if (len < 0 || len > p.maxlen || len > T) {
-        if (leader && tid == 0) latch_error(p.err, STREE_ERR_BAD_PATH, b, -1, len);
-        return;
-    }
-
-    // Round two, all at once: the checks of every path position (depth, the
-    // leaf's ancestor bit), dt at the path's nodes, and the first chunk's B rows
-    // and x values (node ids clamped into range; an invalid path discards them).
-    const int leaf = len > 0 ? pn[len - 1] : 0;
-    const bool leaf_ok = leaf >= 0 && leaf < T;
-    int bad = 0;
-    for (int q = tid; q < len; q += kCThreads) {
-        const int j = pn[q];
-        const bool in = leaf_ok && j >= 0 && j < T;
-        const bool good = in && ((p.tree.anc[((size_t)b * T + leaf) * W + (j >> 5)] >> (j & 31)) & 1u) &&
-                          p.tree.depth[(size_t)b * T + j] == q;
-        if (!good) {
-            bad = 1;
-            atomicMin(&s_badq, q);
-        }
-        dq[q] = in ? load_as_float(p.dt, ((size_t)b * T + j) * H + h, p.dtype) : 0.f;
-    }
-    stage_path_rows(p, Bq, cfq, pn, 0, min(kQChunk, len), b, h, g, p0, rows);
-    // The slab into registers (from L2 by now), issued after the small loads so
-    // that they are not queued behind it.
-    const float4 *src = reinterpret_cast<const float4 *>(slab);
+    // The slab first: h0 is an input of the scan, complete before the prep launch.
+    const float4 *src = reinterpret_cast<const float4 *>(p.h0 + (((size_t)b * H + h) * P + p0) * N);
     float4 hv[kCVec];
 #pragma unroll
     for (int k = 0; k < kCVec; ++k) {
@@ -143,34 +165,26 @@ __global__ void __launch_bounds__(kCThreads, 4) commit_kernel(const CommitParams
                          : "l"(src + f)
                          : "memory");
     }
-    if (__syncthreads_or(bad)) {
-        if (leader && tid == 0) latch_error(p.err, STREE_ERR_BAD_PATH, b, s_badq, pn[s_badq]);
-        return;
-    }
-    const float Ah = s_A;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) {
-        // L along the path (a prefix sum), then the replay weights.
-        float s = 0.f;
-        for (int q = 0; q < len; ++q) {
-            s += dq[q];
-            wq[q] = Ah * s;
-        }
+        s_len = p.ws.len[b];
+        s_alpha = p.ws.alpha[(size_t)b * H + h];
+    }
+    if (tid < p.Lc) {
+        pn[tid] = p.ws.pn[(size_t)b * p.Lc + tid];
+        wq[tid] = p.ws.w[((size_t)b * H + h) * p.Lc + tid];
     }
     __syncthreads();
-    const float Lleaf = len > 0 ? wq[len - 1] : 0.f;
-    __syncthreads();
-    for (int q = tid; q < len; q += kCThreads) wq[q] = expf(Lleaf - wq[q]) * dq[q];
-    const float al = len > 0 ? expf(Lleaf) : 1.f;
-
+    const int len = s_len;
+    if (len < 0) return;                             // invalid tree or path: h_new untouched
+    const float al = s_alpha;
     float4 acc[kCVec];
 #pragma unroll
     for (int k = 0; k < kCVec; ++k) acc[k] = make_float4(al * hv[k].x, al * hv[k].y, al * hv[k].z, al * hv[k].w);
     for (int q0 = 0; q0 < len; q0 += kQChunk) {
         const int nq = min(kQChunk, len - q0);
-        if (q0 > 0) {
-            __syncthreads();
-            stage_path_rows(p, Bq, cfq, pn, q0, nq, b, h, g, p0, rows);
-        }
+        if (q0 > 0) __syncthreads();
+        stage_path_rows(p, Bq, cfq, pn, q0, nq, b, h, g, p0, rows);
         __syncthreads();
 #pragma unroll
         for (int k = 0; k < kCVec; ++k) {
@@ -201,11 +215,22 @@ __global__ void __launch_bounds__(kCThreads, 4) commit_kernel(const CommitParams
 bool commit_supported(const ScanArgs &a)
 {
     if (a.N % 4 != 0 || a.N > kMaxDim || a.P > kMaxDim || a.T > kMaxNodes) return false;
-    const int R = kSlabFloats / a.N;
-    return R >= 1;
+    return kSlabFloats / a.N >= 1;
 }
 
-cudaError_t launch_commit(const ScanArgs &a, cudaStream_t s)
+size_t commit_work_floats(const ScanArgs &a)
+{
+    const size_t Lc = (size_t)(a.maxlen < a.T ? a.maxlen : a.T);
+    return (size_t)a.batch * a.H * (Lc + 1);
+}
+
+size_t commit_work_ints(const ScanArgs &a)
+{
+    const size_t Lc = (size_t)(a.maxlen < a.T ? a.maxlen : a.T);
+    return (size_t)a.batch * (Lc + 1);
+}
+
+cudaError_t launch_commit(const ScanArgs &a, const CommitWork &ws, cudaStream_t s)
 {
     if (a.batch == 0) return cudaSuccess;
     if (!commit_supported(a)) return cudaErrorNotSupported;
@@ -213,8 +238,10 @@ cudaError_t launch_commit(const ScanArgs &a, cudaStream_t s)
     p.x = a.x; p.dt = a.dt; p.B = a.B; p.A = a.A; p.h0 = a.h0;
     p.tree = a.tree;
     p.path = a.path; p.path_len = a.path_len; p.maxlen = a.maxlen;
+    p.Lc = a.maxlen < a.T ? a.maxlen : a.T;
     p.h_new = a.h_new;
     p.err = a.err;
+    p.ws = ws;
     p.T = a.T; p.H = a.H; p.P = a.P; p.N = a.N; p.G = a.G;
     p.dtype = a.dtype;
     p.R = kSlabFloats / a.N;
@@ -222,8 +249,19 @@ cudaError_t launch_commit(const ScanArgs &a, cudaStream_t s)
     p.chunks = (a.P + p.R - 1) / p.R;
     const long long grid = (long long)a.batch * a.H * p.chunks;
     if (grid > 0x7fffffffLL) return cudaErrorNotSupported;
-    commit_kernel<<<(unsigned)grid, kCThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    commit_prep_kernel<<<a.batch, kCThreads, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kCThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, commit_stream_kernel, p);
 }
 
 }  // namespace stree

@@ -18,10 +18,11 @@
 // of 1024 threads per sequence keeps the current p (fp32, the residuals
 // included) in shared memory -- up to 53,248 tokens, 208 KB -- and streams the
 // logits rows of the visited nodes from HBM (a draft row is read once for its
-// softmax statistics, then again from L2 by each residual).  Passes are
-// coalesced element loops with block reductions of (max, sum) pairs; the bonus
-// draw is a block prefix sum over contiguous per-thread chunks.  All arithmetic
-// is fp32.
+// softmax statistics, then again from L2 by each residual).  Each pass walks
+// the row in 16-byte chunks per thread (when rows are 16-byte aligned), unrolled
+// so that several chunk loads are in flight, with block reductions of (max, sum)
+// pairs; the bonus draw is a block prefix sum over contiguous per-thread chunks.
+// All arithmetic is fp32.
 #include <mutex>
 
 #include "stree_internal.cuh"
@@ -33,6 +34,37 @@ constexpr int kSThreads = 1024;
 constexpr int kSWarps = kSThreads / 32;
 constexpr int kMaxVocabSmem = 53248;
 constexpr int kMaxDevices = 64;
+
+// kE consecutive logits starting at v (one 16-byte load when kE > 1: the row
+// start and v are then multiples of 16 bytes).
+template <int kE>
+__device__ __forceinline__ void ld_chunk(const float *r, int v, float (&out)[kE])
+{
+    if constexpr (kE == 4) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(r + v));
+        out[0] = x.x; out[1] = x.y; out[2] = x.z; out[3] = x.w;
+    } else {
+#pragma unroll
+        for (int e = 0; e < kE; ++e) out[e] = __ldg(r + v + e);
+    }
+}
+template <int kE>
+__device__ __forceinline__ void ld_chunk(const __nv_bfloat16 *r, int v, float (&out)[kE])
+{
+    if constexpr (kE == 8) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(r + v));
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h[e]);
+            out[2 * e] = f.x;
+            out[2 * e + 1] = f.y;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < kE; ++e) out[e] = __bfloat162float(r[v + e]);
+    }
+}
 
 __device__ __forceinline__ float ld_logit(const float *r, int v) { return __ldg(r + v); }
 __device__ __forceinline__ float ld_logit(const __nv_bfloat16 *r, int v) { return __bfloat162float(r[v]); }
@@ -65,18 +97,26 @@ __device__ __forceinline__ void merge_ms(float &m, float &s, float m2, float s2)
 }
 
 // Max and sum of exp(z - max) over z_v = row[v] * inv_t; every thread gets both.
-template <typename E>
+// Each thread takes chunks of kE consecutive values, the loop unrolled so that
+// several chunk loads are in flight at once.
+template <typename E, int kE>
 __device__ __forceinline__ void row_stats(const E *row, int V, float inv_t, Red &red, float &m, float &s)
 {
     m = -INFINITY;
     s = 0.f;
-    for (int v = threadIdx.x; v < V; v += kSThreads) {
-        const float z = ld_logit(row, v) * inv_t;
-        if (z > m) {
-            s = (m == -INFINITY ? 0.f : s * __expf(m - z)) + 1.f;
-            m = z;
-        } else {
-            s += __expf(z - m);
+#pragma unroll 4
+    for (int v0 = threadIdx.x * kE; v0 < V; v0 += kSThreads * kE) {
+        float z[kE];
+        ld_chunk<kE>(row, v0, z);
+#pragma unroll
+        for (int e = 0; e < kE; ++e) {
+            const float ze = z[e] * inv_t;
+            if (ze > m) {
+                s = (m == -INFINITY ? 0.f : s * __expf(m - ze)) + 1.f;
+                m = ze;
+            } else {
+                s += __expf(ze - m);
+            }
         }
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -95,17 +135,23 @@ __device__ __forceinline__ void row_stats(const E *row, int V, float inv_t, Red 
 }
 
 // p = softmax(row * inv_t) into shared memory.
-template <typename E>
+template <typename E, int kE>
 __device__ __forceinline__ void load_softmax(const E *row, int V, float inv_t, float *p, Red &red)
 {
     float m, s;
-    row_stats(row, V, inv_t, red, m, s);
+    row_stats<E, kE>(row, V, inv_t, red, m, s);
     const float inv = 1.f / s;
-    for (int v = threadIdx.x; v < V; v += kSThreads) p[v] = __expf(ld_logit(row, v) * inv_t - m) * inv;
+#pragma unroll 4
+    for (int v0 = threadIdx.x * kE; v0 < V; v0 += kSThreads * kE) {
+        float z[kE];
+        ld_chunk<kE>(row, v0, z);
+#pragma unroll
+        for (int e = 0; e < kE; ++e) p[v0 + e] = __expf(z[e] * inv_t - m) * inv;
+    }
     __syncthreads();
 }
 
-template <typename E>
+template <typename E, int kE>
 __global__ void __launch_bounds__(kSThreads, 1)
 accept_sampling_kernel(const E *__restrict__ tl, const E *__restrict__ dl, int V, const int32_t *__restrict__ tokens,
                        const int32_t *__restrict__ parent, int T, float inv_t, const float *__restrict__ u_accept,
@@ -149,13 +195,13 @@ accept_sampling_kernel(const E *__restrict__ tl, const E *__restrict__ dl, int V
     const E *trow0 = tl + (size_t)s * T * V, *drow0 = dl + (size_t)s * T * V;
     int cur = 0, len = 1;
     if (tid == 0) out[0] = 0;
-    load_softmax(trow0, V, inv_t, p, red);
+    load_softmax<E, kE>(trow0, V, inv_t, p, red);
     while (true) {
         int next = -1;
         if (len < maxlen) {
             const E *drow = drow0 + (size_t)cur * V;
             float mq, sq;
-            row_stats(drow, V, inv_t, red, mq, sq);
+            row_stats<E, kE>(drow, V, inv_t, red, mq, sq);
             const float inv_sq = 1.f / sq;
             for (int c = cur + 1; c < T; ++c) {             // children follow their parent
                 if (par[c] != cur) continue;
@@ -167,13 +213,24 @@ accept_sampling_kernel(const E *__restrict__ tl, const E *__restrict__ dl, int V
                 }
                 // Rejected: p <- max(p - q, 0), renormalised (unchanged if all zero).
                 float r = 0.f;
-                for (int v = tid; v < V; v += kSThreads)
-                    r += fmaxf(p[v] - __expf(ld_logit(drow, v) * inv_t - mq) * inv_sq, 0.f);
+#pragma unroll 4
+                for (int v0 = tid * kE; v0 < V; v0 += kSThreads * kE) {
+                    float z[kE];
+                    ld_chunk<kE>(drow, v0, z);
+#pragma unroll
+                    for (int e = 0; e < kE; ++e) r += fmaxf(p[v0 + e] - __expf(z[e] * inv_t - mq) * inv_sq, 0.f);
+                }
                 r = block_sum(r, red);
                 if (r > 0.f) {
                     const float inv_r = 1.f / r;
-                    for (int v = tid; v < V; v += kSThreads)
-                        p[v] = fmaxf(p[v] - __expf(ld_logit(drow, v) * inv_t - mq) * inv_sq, 0.f) * inv_r;
+#pragma unroll 4
+                    for (int v0 = tid * kE; v0 < V; v0 += kSThreads * kE) {
+                        float z[kE];
+                        ld_chunk<kE>(drow, v0, z);
+#pragma unroll
+                        for (int e = 0; e < kE; ++e)
+                            p[v0 + e] = fmaxf(p[v0 + e] - __expf(z[e] * inv_t - mq) * inv_sq, 0.f) * inv_r;
+                    }
                 }
                 __syncthreads();
             }
@@ -182,7 +239,7 @@ accept_sampling_kernel(const E *__restrict__ tl, const E *__restrict__ dl, int V
         if (tid == 0) out[len] = next;
         cur = next;
         ++len;
-        load_softmax(trow0 + (size_t)cur * V, V, inv_t, p, red);
+        load_softmax<E, kE>(trow0 + (size_t)cur * V, V, inv_t, p, red);
     }
     // Bonus token: inverse CDF of p over contiguous per-thread chunks.
     const int chunk = (V + kSThreads - 1) / kSThreads;
@@ -235,10 +292,13 @@ cudaError_t prepare()
     std::lock_guard<std::mutex> lock(g_mutex);
     if (g_prepared[dev]) return cudaSuccess;
     const int bytes = kMaxVocabSmem * (int)sizeof(float);
-    if ((e = cudaFuncSetAttribute(accept_sampling_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bytes)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(accept_sampling_kernel<__nv_bfloat16>,
+    if ((e = cudaFuncSetAttribute(accept_sampling_kernel<float, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(accept_sampling_kernel<float, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(accept_sampling_kernel<__nv_bfloat16, 1>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(accept_sampling_kernel<__nv_bfloat16, 8>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
         return e;
     g_prepared[dev] = true;
@@ -277,14 +337,31 @@ extern "C" stree_status stree_accept_sampling(const void *target_logits, const v
     if (err_out && cudaMemsetAsync(err_out, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return STREE_ERR_CUDA;
     const size_t smem = (size_t)vocab * sizeof(float);
     const float inv_t = 1.f / temperature;
-    if (logit_dtype == STREE_BF16)
-        accept_sampling_kernel<__nv_bfloat16><<<batch, kSThreads, smem, s>>>(
-            static_cast<const __nv_bfloat16 *>(target_logits), static_cast<const __nv_bfloat16 *>(draft_logits), vocab,
-            draft_tokens, parent, n_nodes, inv_t, u_accept, u_bonus, maxlen, accepted_path, path_len, bonus_token,
-            err_out);
-    else
-        accept_sampling_kernel<float><<<batch, kSThreads, smem, s>>>(
-            static_cast<const float *>(target_logits), static_cast<const float *>(draft_logits), vocab, draft_tokens,
-            parent, n_nodes, inv_t, u_accept, u_bonus, maxlen, accepted_path, path_len, bonus_token, err_out);
+    // 16-byte chunk loads when every row starts on a 16-byte boundary.
+    const bool vec = (reinterpret_cast<uintptr_t>(target_logits) & 15u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(draft_logits) & 15u) == 0 && ((size_t)vocab * es) % 16 == 0;
+    if (logit_dtype == STREE_BF16) {
+        const __nv_bfloat16 *t = static_cast<const __nv_bfloat16 *>(target_logits);
+        const __nv_bfloat16 *d = static_cast<const __nv_bfloat16 *>(draft_logits);
+        if (vec)
+            accept_sampling_kernel<__nv_bfloat16, 8><<<batch, kSThreads, smem, s>>>(
+                t, d, vocab, draft_tokens, parent, n_nodes, inv_t, u_accept, u_bonus, maxlen, accepted_path, path_len,
+                bonus_token, err_out);
+        else
+            accept_sampling_kernel<__nv_bfloat16, 1><<<batch, kSThreads, smem, s>>>(
+                t, d, vocab, draft_tokens, parent, n_nodes, inv_t, u_accept, u_bonus, maxlen, accepted_path, path_len,
+                bonus_token, err_out);
+    } else {
+        const float *t = static_cast<const float *>(target_logits);
+        const float *d = static_cast<const float *>(draft_logits);
+        if (vec)
+            accept_sampling_kernel<float, 4><<<batch, kSThreads, smem, s>>>(
+                t, d, vocab, draft_tokens, parent, n_nodes, inv_t, u_accept, u_bonus, maxlen, accepted_path, path_len,
+                bonus_token, err_out);
+        else
+            accept_sampling_kernel<float, 1><<<batch, kSThreads, smem, s>>>(
+                t, d, vocab, draft_tokens, parent, n_nodes, inv_t, u_accept, u_bonus, maxlen, accepted_path, path_len,
+                bonus_token, err_out);
+    }
     return cudaGetLastError() == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
 }

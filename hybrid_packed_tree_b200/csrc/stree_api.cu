@@ -19,6 +19,10 @@ struct stree_ctx {
     // C.B pair scratch
     float *cb = nullptr;
     size_t cap_cb = 0;
+    // stand-alone commit workspace
+    float *cw = nullptr;
+    int32_t *ci = nullptr;
+    size_t cap_cw = 0, cap_ci = 0;
     // error word {status, sequence, position, detail}
     int32_t *err = nullptr;
     // inputs recorded by the last scan, for stree_commit
@@ -249,6 +253,8 @@ stree_status stree_ctx_destroy(stree_ctx *c)
     cudaFree(c->depth);
     cudaFree(c->ok);
     cudaFree(c->cb);
+    cudaFree(c->cw);
+    cudaFree(c->ci);
     cudaFree(c->err);
     delete c;
     return STREE_OK;
@@ -347,8 +353,20 @@ stree_status stree_commit(stree_ctx *c, const int32_t *path, const int32_t *path
     a.tree = tree_view(c);
     a.err = c->err;
     if (a.batch == 0) return STREE_OK;
+    if (commit_supported(a)) {
+        const size_t nf = commit_work_floats(a), ni = commit_work_ints(a);
+        if ((st = ensure(&c->cw, &c->cap_cw, nf)) != STREE_OK) return st;
+        if ((st = ensure(&c->ci, &c->cap_ci, ni)) != STREE_OK) return st;
+        const size_t Lc = (size_t)(a.maxlen < a.T ? a.maxlen : a.T);
+        CommitWork ws;
+        ws.w = c->cw;
+        ws.alpha = c->cw + (size_t)a.batch * a.H * Lc;
+        ws.pn = c->ci;
+        ws.len = c->ci + (size_t)a.batch * Lc;
+        c->launches += 2;
+        return cuda_status(launch_commit(a, ws, static_cast<cudaStream_t>(stream)));
+    }
     ++c->launches;
-    if (commit_supported(a)) return cuda_status(launch_commit(a, static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_scan_simt(a, static_cast<cudaStream_t>(stream)));
 }
 

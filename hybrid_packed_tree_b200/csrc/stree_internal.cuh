@@ -75,9 +75,19 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 bool small_supported(const ScanArgs &a);
 cudaError_t launch_scan_small(const ScanArgs &a, cudaStream_t s);
 
-// Commit by replay of the accepted path alone (no tree term, no root term).
+// Commit by replay of the accepted path alone (no tree term, no root term).  Its
+// workspace: per sequence the path's nodes and length, per (sequence, head) the
+// replay weights and exp(L_leaf).  Sizes in floats / ints from the two helpers.
+struct CommitWork {
+    float *w;          // [batch, H, Lc]
+    float *alpha;      // [batch, H]
+    int32_t *pn;       // [batch, Lc]
+    int32_t *len;      // [batch]
+};
 bool commit_supported(const ScanArgs &a);
-cudaError_t launch_commit(const ScanArgs &a, cudaStream_t s);
+size_t commit_work_floats(const ScanArgs &a);
+size_t commit_work_ints(const ScanArgs &a);
+cudaError_t launch_commit(const ScanArgs &a, const CommitWork &ws, cudaStream_t s);
 
 // Resolves a kernel selection against the shape; false when the selection
 // cannot run it (STREE_ERR_UNSUPPORTED).

@@ -336,6 +336,34 @@ stree_status stree_gdn_tree_scan_commit(const void *q, const void *k, const void
                                         float *S_new, int32_t *err_out, void *stream);
 
 /*
+ * Tree-masked attention of the hybrid model's Transformer layers over the packed
+ * tree (STree abstract: hybrid SSM and Transformer layers; STree summary,
+ * "Approach": the packed tree sequence with a tree mask).  Node i, query head h
+ * (key/value head g = h / (heads_q / heads_kv)) attends to the valid context and
+ * to its own root path:
+ *     o[b,i,h] = sum_j softmax_j(scale q[b,i,h] . k_j) v_j,
+ *     j over k_ctx/v_ctx[b, 0 .. ctx_len[b]-1, g] and k_tree/v_tree[b, anc(i), g].
+ *
+ *   q, o          [batch, n_nodes, heads_q, 128]  bf16
+ *   k_ctx, v_ctx  [batch, ctx_cap, heads_kv, 128] bf16 (the cache; positions past
+ *                 ctx_len[b] are never used, whatever they hold)
+ *   k_tree, v_tree [batch, n_nodes, heads_kv, 128] bf16 (the tree's own keys and values)
+ *   ctx_len       [batch] int32, clamped to [0, ctx_cap]
+ *   parent        [batch, n_nodes] int32: the packed tree (as for the scan)
+ *   err_out       device int32[4] error word of this call (cleared by the call); required
+ *
+ * fp32 accumulation and softmax; P rounded to bf16 for the second product.
+ * Shapes: head dim 128, n_nodes up to 128, heads_q / heads_kv dividing 128
+ * (else STREE_ERR_UNSUPPORTED); scale > 0.  An invalid tree latches
+ * STREE_ERR_BAD_TREE and leaves that sequence's o untouched.  The caller owns
+ * every buffer; the call allocates nothing and runs on `stream`.
+ */
+stree_status stree_tree_attention(const void *q, const void *k_ctx, const void *v_ctx, const void *k_tree,
+                                  const void *v_tree, const int32_t *ctx_len, const int32_t *parent, int n_nodes,
+                                  int batch, int ctx_cap, int heads_q, int heads_kv, int head_dim, float scale,
+                                  stree_dtype dtype, void *o, int32_t *err_out, void *stream);
+
+/*
  * Resolve accepted paths against the context's current tree: leaf_out[b] (device
  * int32 [batch]) receives the last node of a valid path, -1 for an empty path and
  * -2 for an invalid one (which also latches STREE_ERR_BAD_PATH).
