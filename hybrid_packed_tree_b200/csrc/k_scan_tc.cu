@@ -88,6 +88,7 @@ struct TcParams {
     int fault;                             // test hook: 1 withholds the first tile's coefficient hand-off
     int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, pre, bs_mh, tc_commit, hpt, pair_cap,
         acc_cols, cm_col;
+    int tpg, sw_milli;                     // tiles per (sequence, group); cost of a switch in tiles x 1000
     uint32_t tmem_cols;
     uint32_t off_x, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_coef, coef_slot,
         off_pnode, off_praw, off_par, off_dep, off_bs, off_cf, off_bt, off_bar, off_misc, off_ad, off_pcb, off_pj,
@@ -372,8 +373,23 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
 
     const uint32_t h0_stage_bytes = (uint32_t)RB * 512u;
     const uint32_t tx_bytes = h0_stage_bytes + (uint32_t)T * RB * 2u;
-    const int start = (int)((long long)blockIdx.x * p.ntiles / gridDim.x);
-    const int end = (int)((long long)(blockIdx.x + 1) * p.ntiles / gridDim.x);
+    // Tile range of this CTA: equal shares of a cost line on which every tile costs
+    // one unit and every (sequence, group) start costs sw_milli / 1000 more (the
+    // switch), so that a range crossing a group boundary takes fewer tiles.
+    int start, end;
+    {
+        const long long per = (long long)p.tpg * 1000 + p.sw_milli;
+        const long long total = (long long)(p.ntiles / p.tpg) * per;
+        auto tile_at = [&](long long c) -> int {
+            if (c >= total) return p.ntiles;
+            const long long q = c / per, r = c - q * per;
+            long long t = q * p.tpg + (r <= p.sw_milli ? 0 : (r - p.sw_milli + 999) / 1000);
+            if (t > (q + 1) * p.tpg) t = (q + 1) * p.tpg;
+            return (int)t;
+        };
+        start = tile_at((long long)blockIdx.x * total / gridDim.x);
+        end = tile_at((long long)(blockIdx.x + 1) * total / gridDim.x);
+    }
     // With p.pre the first S tiles are requested before anything else, once the
     // preceding grid (the kernel is a programmatic dependent) has completed.
     const uint32_t npre = p.pre ? (uint32_t)min(S, end - start) : 0u;
@@ -422,6 +438,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     };
 
     if (p.pre) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // A later launch on the stream (the next layer) may be scheduled onto SMs as
+    // this grid's CTAs leave; it waits for this grid's completion before it reads
+    // anything, so only its set-up overlaps this grid's tail.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         ptx::prefetch_tensormap(&tm_h0);
         ptx::prefetch_tensormap(&tm_x);
@@ -1301,6 +1321,8 @@ bool plan(const ScanArgs &a, TcPlan &pl)
     best.G = a.G;
     best.tps = a.H * a.P / chosen;
     best.ntiles = a.batch * best.tps;
+    best.tpg = (a.H / a.G) * a.P / chosen;          // whole tiles: rb_valid keeps groups tile-aligned
+    best.sw_milli = 1500;                           // a switch costs about one and a half tiles
     pl.p = best;
     pl.smem = best_smem;
     return true;
