@@ -41,7 +41,7 @@ EXPORTS = (
     "stree_build_tree",
     "stree_tree_scan", "stree_commit", "stree_tree_scan_commit", "stree_tree_scan_commit_noalloc",
     "stree_resolve_path", "stree_unrolled_scan", "stree_accept_greedy", "stree_accept_sampling",
-    "stree_gdn_tree_scan_commit", "stree_tree_attention",
+    "stree_gdn_tree_scan_commit", "stree_tree_attention", "stree_tree_attention_workspace_size",
     "stree_sync_check", "stree_status_string", "stree_version",
 )
 
@@ -64,7 +64,8 @@ _lib.stree_accept_greedy.argtypes = [_vp, _i, _i, _vp, _vp, _i, _i, _i, _vp, _vp
 _lib.stree_accept_sampling.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _i, _i, ctypes.c_float, _vp, _vp, _i, _vp,
                                         _vp, _vp, _vp, _vp]
 _lib.stree_gdn_tree_scan_commit.argtypes = [_vp] * 7 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp, _vp]
-_lib.stree_tree_attention.argtypes = [_vp] * 7 + [_i] * 6 + [ctypes.c_float, _i, _vp, _vp, _vp]
+_lib.stree_tree_attention.argtypes = [_vp] * 7 + [_i] * 6 + [ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp, _vp]
+_lib.stree_tree_attention_workspace_size.argtypes = [_i] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
 _lib.stree_sync_check.argtypes = [_vp, _vp, _ip]
 _lib.stree_status_string.argtypes = [_i]
 _lib.stree_status_string.restype = ctypes.c_char_p
@@ -328,19 +329,32 @@ def stree_gdn_tree_scan_commit(q, k, v, alpha, beta, S0, parent, o, path=None, p
     return o, S_new
 
 
-def stree_tree_attention(q, k_ctx, v_ctx, k_tree, v_tree, ctx_len, parent, o, scale, err_out, stream=None):
+def stree_tree_attention_workspace_size(n_nodes, batch, ctx_cap, heads_q, heads_kv, head_dim=128) -> int:
+    """Bytes of the workspace stree_tree_attention splits into on the current device (0: no split)."""
+    n = ctypes.c_size_t(0)
+    _check(_lib.stree_tree_attention_workspace_size(int(n_nodes), int(batch), int(ctx_cap), int(heads_q),
+                                                    int(heads_kv), int(head_dim), ctypes.byref(n)),
+           "stree_tree_attention_workspace_size")
+    return int(n.value)
+
+
+def stree_tree_attention(q, k_ctx, v_ctx, k_tree, v_tree, ctx_len, parent, o, scale, err_out, workspace=None,
+                         stream=None):
     """Tree-masked attention: o [b, T, Hq, 128] (bf16) from q [b, T, Hq, 128], the
     context cache k_ctx / v_ctx [b, S, Hkv, 128] (S may be 0), the tree's own k_tree /
-    v_tree [b, T, Hkv, 128], ctx_len [b] and parent [b, T]."""
+    v_tree [b, T, Hkv, 128], ctx_len [b] and parent [b, T].  workspace: a device
+    uint8 tensor of stree_tree_attention_workspace_size() bytes, or None (no split)."""
     batch, T, Hq, d = q.shape
     S, Hkv = k_ctx.shape[1], k_ctx.shape[2]
     bf = (torch.bfloat16,)
+    ws = _ptr(workspace, "workspace", (torch.uint8,)) if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
     st = _lib.stree_tree_attention(_ptr(q, "q", bf), _ptr(k_ctx, "k_ctx", bf) if S else None,
                                    _ptr(v_ctx, "v_ctx", bf) if S else None, _ptr(k_tree, "k_tree", bf),
                                    _ptr(v_tree, "v_tree", bf), _ptr(ctx_len, "ctx_len", (torch.int32,)),
                                    _ptr(parent, "parent", (torch.int32,)), T, batch, S, Hq, Hkv, d, float(scale),
-                                   STREE_BF16, _ptr(o, "o", bf), _ptr(err_out, "err_out", (torch.int32,)),
-                                   _stream(stream))
+                                   STREE_BF16, _ptr(o, "o", bf), ws, ws_bytes,
+                                   _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))
     _check(st, "stree_tree_attention")
     return o
 

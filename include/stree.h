@@ -69,6 +69,7 @@
 #define STREE_H
 
 #include <stdint.h>
+#include <stddef.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -350,9 +351,16 @@ stree_status stree_gdn_tree_scan_commit(const void *q, const void *k, const void
  *   k_tree, v_tree [batch, n_nodes, heads_kv, 128] bf16 (the tree's own keys and values)
  *   ctx_len       [batch] int32, clamped to [0, ctx_cap]
  *   parent        [batch, n_nodes] int32: the packed tree (as for the scan)
+ *   workspace     device scratch of at least stree_tree_attention_workspace_size()
+ *                 bytes, 16-byte aligned, or NULL; owned by the caller, overwritten
  *   err_out       device int32[4] error word of this call (cleared by the call); required
  *
  * fp32 accumulation and softmax; P rounded to bf16 for the second product.
+ * With few query tiles and a long context the key blocks are split over several
+ * CTAs whose partial outputs go to the workspace and are merged by a second
+ * launch on the same stream; with workspace NULL or too small the call runs one
+ * CTA per query tile (same result up to rounding order, slower on long contexts).
+ * Two calls that share a workspace must be ordered (same stream).
  * Shapes: head dim 128, n_nodes up to 128, heads_q / heads_kv dividing 128
  * (else STREE_ERR_UNSUPPORTED); scale > 0.  An invalid tree latches
  * STREE_ERR_BAD_TREE and leaves that sequence's o untouched.  The caller owns
@@ -361,7 +369,16 @@ stree_status stree_gdn_tree_scan_commit(const void *q, const void *k, const void
 stree_status stree_tree_attention(const void *q, const void *k_ctx, const void *v_ctx, const void *k_tree,
                                   const void *v_tree, const int32_t *ctx_len, const int32_t *parent, int n_nodes,
                                   int batch, int ctx_cap, int heads_q, int heads_kv, int head_dim, float scale,
-                                  stree_dtype dtype, void *o, int32_t *err_out, void *stream);
+                                  stree_dtype dtype, void *o, void *workspace, size_t workspace_bytes,
+                                  int32_t *err_out, void *stream);
+
+/*
+ * Workspace bytes that stree_tree_attention wants for these shapes on the current
+ * device (its split plan depends on the device's SM count); 0 when it does not
+ * split.  Same shape rules as stree_tree_attention (STREE_ERR_UNSUPPORTED).
+ */
+stree_status stree_tree_attention_workspace_size(int n_nodes, int batch, int ctx_cap, int heads_q, int heads_kv,
+                                                 int head_dim, size_t *bytes);
 
 /*
  * Resolve accepted paths against the context's current tree: leaf_out[b] (device

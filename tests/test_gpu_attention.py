@@ -2,7 +2,8 @@
 by element at the bf16 tolerance (2e-2 max|ref|): trees of the workloads with
 ragged context lengths (including none), grouped heads of several sizes, the
 128-node chain, cache positions past the valid length holding NaN (never read),
-and an invalid tree."""
+and an invalid tree; each case both split over CTAs (partials in a workspace,
+merged by a second launch) and unsplit (no workspace)."""
 import numpy as np
 import pytest
 import torch
@@ -27,12 +28,21 @@ def _bf16(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def _run(st, a):
+def _workspace(st, a, split, short=0):
+    if not split:
+        return None
+    b, T, hq, _ = a["q"].shape
+    n = st.stree_tree_attention_workspace_size(T, b, a["k_ctx"].shape[1], hq, a["k_ctx"].shape[2])
+    return torch.full((max(n - short, 0),), 0xFF, dtype=torch.uint8, device="cuda")   # NaN-filled partials
+
+
+def _run(st, a, split=True, short=0):
     q = _bf16(a["q"])
     o = torch.full_like(q, 7.0)
     err = torch.full((4,), -1, dtype=torch.int32, device="cuda")
     st.stree_tree_attention(q, _bf16(a["k_ctx"]), _bf16(a["v_ctx"]), _bf16(a["k_tree"]), _bf16(a["v_tree"]),
-                            i32(a["ctx_len"]), i32(a["parent"]), o, a["scale"], err)
+                            i32(a["ctx_len"]), i32(a["parent"]), o, a["scale"], err,
+                            workspace=_workspace(st, a, split, short))
     torch.cuda.synchronize()
     return o, err.tolist()
 
@@ -51,16 +61,43 @@ CASES = [
     ("m2_2p7b", None, 384, [383], 32, 4),
     ("hyb8b", 2, 256, [256, 100], 8, 8),
     ("wide256_chain", 1, 256, [200], 16, 16),
+    ("hyb8b", 1, 4096, [4096], 32, 8),                 # 33 key blocks over many splits
+    ("serve64", 2, 2048, [2047, 129], 64, 8),          # two query tiles per head group
 ]
 
 
+@pytest.mark.parametrize("split", [True, False], ids=["split", "unsplit"])
 @pytest.mark.parametrize("name,batch,cap,lens,hq,hkv", CASES)
-def test_tree_attention_matches_oracle(st, name, batch, cap, lens, hq, hkv):
+def test_tree_attention_matches_oracle(st, name, batch, cap, lens, hq, hkv, split):
     w = wl.make_workload(name, batch=batch, layers=1)
     a = wl.attention_inputs(w.parent, cap, lens, heads_q=hq, heads_kv=hkv, seed=61)
-    o, err = _run(st, a)
+    o, err = _run(st, a, split)
     assert err == [0, 0, 0, 0]
     assert_close(f64(o), _oracle(a), "bf16", f"{name} o")
+
+
+def test_tree_attention_workspace_sizes(st):
+    # A long context over few tiles splits; many tiles over a short context do not.
+    assert st.stree_tree_attention_workspace_size(26, 1, 4096, 32, 8) > 0
+    assert st.stree_tree_attention_workspace_size(64, 64, 1024, 32, 8) == 0
+    assert st.stree_tree_attention_workspace_size(26, 0, 4096, 32, 8) == 0
+    with pytest.raises(st.StreeError):
+        st.stree_tree_attention_workspace_size(26, 1, 4096, 32, 8, head_dim=64)
+
+
+def test_tree_attention_workspace_too_small_runs_unsplit(st):
+    w = wl.make_workload("hyb8b", batch=2, layers=1)
+    a = wl.attention_inputs(w.parent, 2048, [2048, 700], heads_q=32, heads_kv=8, seed=64)
+    o_split, err = _run(st, a, split=True)
+    assert err == [0, 0, 0, 0]
+    o_short, err = _run(st, a, split=True, short=16)
+    assert err == [0, 0, 0, 0]
+    o_none, err = _run(st, a, split=False)
+    assert err == [0, 0, 0, 0]
+    assert torch.equal(o_short, o_none)                # the short workspace is not used
+    ref = _oracle(a)
+    assert_close(f64(o_split), ref, "bf16", "split o")
+    assert_close(f64(o_none), ref, "bf16", "unsplit o")
 
 
 def test_tree_attention_without_context(st):
@@ -71,18 +108,19 @@ def test_tree_attention_without_context(st):
     err = torch.full((4,), -1, dtype=torch.int32, device="cuda")
     empty = torch.empty((1, 0, 2, 128), dtype=torch.bfloat16, device="cuda")
     st.stree_tree_attention(q, empty, empty, _bf16(a["k_tree"]), _bf16(a["v_tree"]), i32(a["ctx_len"]),
-                            i32(a["parent"]), o, a["scale"], err)
+                            i32(a["parent"]), o, a["scale"], err, workspace=_workspace(st, a, True))
     torch.cuda.synchronize()
     assert err.tolist() == [0, 0, 0, 0]
     assert_close(f64(o), _oracle(a), "bf16", "o")
 
 
-def test_tree_attention_invalid_tree(st):
+@pytest.mark.parametrize("split", [True, False], ids=["split", "unsplit"])
+def test_tree_attention_invalid_tree(st, split):
     par = [-1, 0, 0, 1, 1, 2]
     parent = np.asarray([par, par], np.int32)
     parent[1, 3] = 4
-    a = wl.attention_inputs(parent, 128, [128, 50], heads_q=4, heads_kv=1, seed=63)
-    o, err = _run(st, a)
+    a = wl.attention_inputs(parent, 1024, [1024, 50], heads_q=4, heads_kv=1, seed=63)
+    o, err = _run(st, a, split)
     assert err[0] == 3 and err[1] == 1
     assert torch.all(o[1] == 7.0)
     assert_close(f64(o[:1]), _oracle(a, keep=[0]), "bf16", "o of the valid sequence")
