@@ -133,7 +133,9 @@ extern "C" stree_status stree_tree_scan_commit_noalloc(
         return STREE_ERR_MISALIGNED;
 
     // Scratch layout: error word, masks, depths, flags, then the C.B pair
-    // scratch when the CUDA-core kernel runs.  Sizes beyond the array are rejected.
+    // scratch of the CUDA-core kernel, or of the tensor-core kernel on trees with
+    // more ancestor pairs than its shared memory holds.  Sizes beyond the array
+    // are rejected (the tensor-core pair scratch is optional).
     const size_t T = (size_t)n_nodes, W = (T + 31) / 32, nb = (size_t)batch;
     const size_t off_err = 0;
     const size_t off_anc = 256;
@@ -150,6 +152,10 @@ extern "C" stree_status stree_tree_scan_commit_noalloc(
     size_t need = off_cb;
     if (path == ScanPath::Simt) need += round256(nb * (size_t)ngroups * T * T * sizeof(float));
     if (need > kNoAllocScratch) return STREE_ERR_UNSUPPORTED;
+    // The tensor-core kernel's pair scratch for deep trees, when it fits (without
+    // it the kernel recomputes those products per tile: same result, slower).
+    const size_t pair_bytes = path == ScanPath::Tc ? round256(tc_pair_scratch_floats(a) * sizeof(float)) : 0;
+    const bool use_pairs = pair_bytes > 0 && off_cb + pair_bytes <= kNoAllocScratch;
 
     int32_t *err = err_out ? err_out : reinterpret_cast<int32_t *>(base + off_err);
     uint32_t *anc = reinterpret_cast<uint32_t *>(base + off_anc);
@@ -170,6 +176,7 @@ extern "C" stree_status stree_tree_scan_commit_noalloc(
     a.tree_ok = ok;
     a.err = err;
     if (path == ScanPath::Simt) a.cb = reinterpret_cast<float *>(base + off_cb);
+    if (use_pairs) a.pair_scratch = reinterpret_cast<float *>(base + off_cb);
     int64_t launches = 0;
     return launch_scan(path, a, s, &launches) == cudaSuccess ? STREE_OK : STREE_ERR_CUDA;
 }

@@ -33,7 +33,9 @@
 // bounded mbarrier waits; a timeout latches STREE_ERR_TIMEOUT and the CTA runs
 // to its end without further work.  Precision: the root term rounds h0 to tf32
 // and the masked decay matrix (D_h on its diagonal included) to bf16 inside the
-// MMAs (fp32 accumulation); the commit and every other step are fp32.
+// MMAs (fp32 accumulation); on trees whose ancestor pairs overflow the fp32 pair
+// table (deep trees: up to three times as many pairs are kept) C_i . B_j is held
+// in bf16 before that product; the commit and every other step are fp32.
 #include <cuda.h>
 
 #include <mutex>
@@ -89,6 +91,8 @@ struct TcParams {
     int T, T_pad, KA, H, P, G, RB, NB, S, tps, ntiles, maxlen, do_commit, pre, bs_mh, tc_commit, hpt, pair_cap,
         acc_cols, cm_col;
     int tpg, sw_milli;                     // tiles per (sequence, group); cost of a switch in tiles x 1000
+    float *pcb_g;                          // trees whose pairs overflow shared memory: C_i . B_j of the
+    int pair_max;                          //   pairs in a global region of pair_max floats per CTA
     uint32_t tmem_cols;
     uint32_t off_x, x_stage, off_c, off_mh, mh_head, off_bp, off_anc, off_poff, off_coef, coef_slot,
         off_pnode, off_praw, off_par, off_dep, off_bs, off_cf, off_bt, off_bar, off_misc, off_ad, off_pcb, off_pj,
@@ -362,6 +366,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
     float *pcb = reinterpret_cast<float *>(smem + p.off_pcb);         // [pair_cap] C_i . B_j
     uint8_t *pj = smem + p.off_pj;                                    // [pair_cap] j
     uint8_t *pi = smem + p.off_pi;                                    // [pair_cap] i
+    // Deep trees whose pairs overflow the fp32 table: the same region as bf16 values
+    // in row order (node i's pairs at poff[i] .., its ancestors in increasing order).
+    __nv_bfloat16 *pcb16 = reinterpret_cast<__nv_bfloat16 *>(smem + p.off_pcb);   // [3 pair_cap]
     const bool b_staged = p.off_bs != 0;
     uint8_t *cfs = smem + p.off_cf;                                   // [RB][8] fp32 commit coefficients (MMA A)
     uint8_t *bts = smem + p.off_bt;                                   // [128][8] fp32 path rows of B^T (MMA B)
@@ -679,7 +686,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     int total = 0;
                     for (int w = 0; w < kWarps; ++w) total += misc[M_WSUM + w];
                     misc[M_TOTAL] = total;
-                    misc[M_INSMEM] = total <= p.pair_cap;
+                    misc[M_INSMEM] = total <= p.pair_cap ? 1 : total <= 3 * p.pair_cap ? 2 : 0;
                 }
                 cur_b = b;
             }
@@ -711,7 +718,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     reinterpret_cast<float4 *>(Bp)[q] = make_float4(b0, b1, b2, b3);
                 }
             }
-            if (misc[M_INSMEM]) {
+            if (misc[M_INSMEM] == 1) {
                 const int total = misc[M_TOTAL];
                 // Node i's pairs: its ancestors in increasing order.
                 for (int i = tid; i < T; i += kThreads) {
@@ -738,6 +745,28 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     v += __shfl_xor_sync(0xffffffffu, v, 1);
                     v += __shfl_xor_sync(0xffffffffu, v, 2);
                     if (part == 0 && q0 < total) pcb[q] = v;
+                }
+            } else if (misc[M_INSMEM] == 2 || p.pcb_g) {
+                // Too many pairs for the fp32 table (deep trees): the products rounded
+                // to bf16 in the same region (row order), else in this CTA's own region
+                // of a global scratch (fp32), read back by the prep warps.
+                const bool h16 = misc[M_INSMEM] == 2;
+                const int total = h16 ? (int)misc[M_TOTAL] : min((int)misc[M_TOTAL], p.pair_max);
+                float *pg = h16 ? nullptr : p.pcb_g + (size_t)blockIdx.x * p.pair_max;
+                const int part = lane & 3;
+                for (int q0 = (tid >> 2); q0 < ((total + 7) & ~7); q0 += kThreads / 4) {
+                    const int q = q0 < total ? q0 : total - 1;
+                    const int i = pair_row(poff, T, q);
+                    const int j = nth_set_bit(ancs + i * W, W, q - poff[i]);
+                    const int rot = (lane >> 2) & 7;
+                    float v = b_staged ? dot_cb_part<true>(cs, T_pad, Bs + j * kDstate, i, part, rot)
+                                       : dot_cb_part<false>(cs, T_pad, Bseq + (size_t)j * brow, i, part, rot);
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    if (part == 0 && q0 < total) {
+                        if (h16) pcb16[q] = __float2bfloat16_rn(v);
+                        else pg[q] = v;
+                    }
                 }
             }
             if (p.bs_mh) {                                     // B rows read: clear the region for M_h
@@ -875,7 +904,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 ok = !misc[M_ABORT];
                 if (ok) {
                     const int total = misc[M_TOTAL];
-                    if (misc[M_INSMEM]) {
+                    if (misc[M_INSMEM] == 1) {
                         for (int q = ptid; q < hpt * total; q += kPrepThreads) {
                             const int hh = q / total, qq = q - hh * total;
                             const int i = pi[qq], j = pj[qq];
@@ -884,13 +913,41 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                             *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
                                 __float2bfloat16_rn(m);
                         }
+                    } else if (misc[M_INSMEM] == 2) {
+                        // Row order: kRowParts threads per (head, node) take every
+                        // kRowParts-th of its ancestors (no per-pair index search).
+                        constexpr int kRowParts = 3;
+                        for (int it = ptid; it < hpt * T * kRowParts; it += kPrepThreads) {
+                            const int hh = it / (T * kRowParts), rem = it - hh * T * kRowParts;
+                            const int i = rem / kRowParts, part = rem - i * kRowParts;
+                            const float Li = Ls[hh * T + i];
+                            int q = poff[i], k = 0;
+                            for (int w = 0; w < W; ++w) {
+                                uint32_t bits = ancs[i * W + w];
+                                while (bits) {
+                                    const int j = (w << 5) + __ffs(bits) - 1;
+                                    bits &= bits - 1;
+                                    if (k == part) {
+                                        float m = expf(Li - Ls[hh * T + j]) * __bfloat162float(pcb16[q]) *
+                                                  dts[hh * T + j];
+                                        if (i == j) m += Dsh[hfirst + hh];
+                                        *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head +
+                                                                           k_off(i, j, T_pad)) = __float2bfloat16_rn(m);
+                                    }
+                                    ++q;
+                                    k = k == kRowParts - 1 ? 0 : k + 1;
+                                }
+                            }
+                        }
                     } else {
+                        const float *pg = p.pcb_g ? p.pcb_g + (size_t)blockIdx.x * p.pair_max : nullptr;
                         for (int q = ptid; q < hpt * total; q += kPrepThreads) {
                             const int hh = q / total, qq = q - hh * total;
                             const int i = pair_row(poff, T, qq);
                             const int j = nth_set_bit(ancs + i * W, W, qq - poff[i]);
-                            float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) *
-                                      dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i) * dts[hh * T + j];
+                            const float cb = pg ? (qq < p.pair_max ? pg[qq] : 0.f)
+                                                : dot_cb(cs, T_pad, Bseq + (size_t)j * brow, i);
+                            float m = expf(Ls[hh * T + i] - Ls[hh * T + j]) * cb * dts[hh * T + j];
                             if (i == j) m += Dsh[hfirst + hh];
                             *reinterpret_cast<__nv_bfloat16 *>(mh + hh * p.mh_head + k_off(i, j, T_pad)) =
                                 __float2bfloat16_rn(m);
@@ -1336,6 +1393,17 @@ bool tc_supported(const ScanArgs &a)
     return plan(a, pl);
 }
 
+size_t tc_pair_scratch_floats(const ScanArgs &a)
+{
+    TcPlan pl;
+    if (!plan(a, pl)) return 0;
+    const long long pairs = (long long)a.T * (a.T + 1) / 2;
+    if (pl.p.pair_cap >= pairs) return 0;
+    long long grid = num_sms();
+    if (grid > pl.p.ntiles) grid = pl.p.ntiles;
+    return (size_t)grid * (size_t)pairs;
+}
+
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
 {
     TcPlan pl;
@@ -1359,6 +1427,10 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s)
     p.wait_ns = a.wait_ns ? a.wait_ns : ptx::kWaitLimitNs;
     p.fault = a.fault;
     p.err = a.err;
+    if (a.pair_scratch && tc_pair_scratch_floats(a) > 0) {
+        p.pcb_g = a.pair_scratch;
+        p.pair_max = a.T * (a.T + 1) / 2;
+    }
 
     EncodeTiledFn enc = encode_fn();
     const int HP = a.H * a.P;

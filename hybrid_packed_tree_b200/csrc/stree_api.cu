@@ -144,6 +144,13 @@ stree_status run_scan(stree_ctx *c, ScanArgs &a, cudaStream_t s)
         stree_status st = ensure(&c->cb, &c->cap_cb, (size_t)a.batch * a.G * a.T * a.T);
         if (st != STREE_OK) return st;
         a.cb = c->cb;
+    } else if (path == ScanPath::Tc) {
+        const size_t nf = tc_pair_scratch_floats(a);
+        if (nf) {
+            stree_status st = ensure(&c->cb, &c->cap_cb, nf);
+            if (st != STREE_OK) return st;
+            a.pair_scratch = c->cb;
+        }
     }
     return cuda_status(launch_scan(path, a, s, &c->launches));
 }

@@ -51,6 +51,8 @@ struct ScanArgs {
     uint32_t *tree_anc;
     int32_t *tree_depth, *tree_ok;
     float *cb;                         // scratch [batch, G, T, T]: C_i . B_j on ancestor pairs
+    float *pair_scratch;               // tensor-core kernel, trees with more ancestor pairs than its
+                                       // shared memory holds: tc_pair_scratch_floats() floats (or NULL)
     int32_t *err;
     unsigned long long wait_ns;        // tensor-core kernel: bounded-wait limit (0: the default)
     int fault;                         // tensor-core kernel: failure-path test hook (0: off)
@@ -70,6 +72,9 @@ cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t s);
 // Tensor-core path: whether the shape is supported, and the launcher.
 bool tc_supported(const ScanArgs &a);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
+// Floats of ScanArgs::pair_scratch the tensor-core kernel uses for this shape
+// (0: every tree's pairs fit in its shared memory).
+size_t tc_pair_scratch_floats(const ScanArgs &a);
 
 // Small-batch path: whether the shape is supported, and the launcher.
 bool small_supported(const ScanArgs &a);

@@ -39,7 +39,8 @@ def _with_ctx(st, d, tr):
     return y, h_new
 
 
-@pytest.mark.parametrize("name,batch", [("tiny", None), ("m2_2p7b", None), ("hyb8b", None), ("serve64", 4)])
+@pytest.mark.parametrize("name,batch", [("tiny", None), ("m2_2p7b", None), ("hyb8b", None), ("serve64", 4),
+                                        ("wide256_chain", 2)])
 def test_noalloc_matches_context_entry_point_twice(st, name, batch):
     w = wl.make_workload(name, batch=batch, layers=1)
     d, tr = upload_layer(w), upload_tree(w)
