@@ -4,7 +4,10 @@ pure-decay closed form at beta = 0, the delta rule's write property (with alpha
 = beta = 1 and a unit key, the new state maps that key exactly to its value),
 exact recall along a path of orthonormal keys, each leaf against its path
 decoded alone, identical siblings, the commit against the leaf's state, the
-packed triangular-solve formulation, and a mutation check.
+packed triangular-solve formulation, and a mutation check.  With the erase
+strength given apart from the write strength: a hand-worked decoupled case, and
+zero erase against the closed form of gated linear attention (every node's output
+a decayed sum over its root path, written out directly).
 """
 import json
 import os
@@ -125,6 +128,46 @@ def test_identical_siblings_and_commit_at_the_leaf():
         np.testing.assert_allclose(S[0, h] @ q[0, 3, 0], o[0, 3, h], rtol=1e-12, atol=1e-12)
 
 
+def test_golden_decoupled_erase_and_write():
+    with open(os.path.join(GOLD, "gdn_decoupled.json")) as f:
+        g = json.load(f)
+    T = len(g["parent"])
+    q = np.asarray(g["q"]).reshape(1, T, 1, 2)
+    k = np.asarray(g["k"]).reshape(1, T, 1, 2)
+    v = np.asarray(g["v"]).reshape(1, T, 1, 1)
+    a, be, er = (np.asarray(g[n]).reshape(1, T, 1) for n in ("alpha", "beta", "erase"))
+    S0 = np.asarray(g["S0"]).reshape(1, 1, 1, 2)
+    parent = np.asarray([g["parent"]])
+    o = oracle_gdn_tree(q, k, v, a, be, S0, parent, erase=er)
+    np.testing.assert_allclose(o.reshape(-1), g["o"], rtol=0, atol=1e-12)
+    for i in range(3):
+        path = np.asarray([[0] if i == 0 else [0, i]])
+        S = oracle_gdn_commit(k, v, a, be, S0, parent, path, np.asarray([path.shape[1]]), erase=er)
+        np.testing.assert_allclose(S.reshape(-1), g["S"][i], rtol=0, atol=1e-12)
+
+
+def test_zero_erase_is_gated_linear_attention():
+    """a = 0: o_i = gamma_i S0 q_i + sum_{j in anc(i)} (gamma_i / gamma_j) beta_j (k_j . q_i) v_j,
+    with gamma the product of alpha over the root path (the closed form, summed here
+    directly instead of walking the recurrence)."""
+    parent = wl.random_tree(np.random.default_rng(11), 14, max_depth=5)[None]
+    q, k, v, a, be, S0 = _rand(12, parent, Hv=4, Hk=2, unit=False)
+    o = oracle_gdn_tree(q, k, v, a, be, S0, parent, erase=np.zeros_like(be))
+    for i in range(14):
+        path = []
+        j = i
+        while j >= 0:
+            path.insert(0, j)
+            j = int(parent[0, j])
+        for h in range(4):
+            g = h // 2
+            gam = np.cumprod(a[0, path, h])                # gamma of each path node
+            ref = gam[-1] * (S0[0, h] @ q[0, i, g])
+            for t, j in enumerate(path):
+                ref = ref + gam[-1] / gam[t] * be[0, j, h] * (k[0, j, g] @ q[0, i, g]) * v[0, j, h]
+            np.testing.assert_allclose(o[0, i, h], ref, rtol=1e-12, atol=1e-12)
+
+
 def test_packed_triangular_solve_equals_the_walk():
     for seed, T, depth in ((9, 20, 6), (10, 40, 12)):
         parent = np.stack([wl.random_tree(np.random.default_rng(seed + s), T, max_depth=depth) for s in range(2)])
@@ -136,29 +179,34 @@ def test_packed_triangular_solve_equals_the_walk():
             nodes = wl.root_path_nodes(parent[s], leaf)
             path[s, :len(nodes)] = nodes
             plen[s] = len(nodes)
-        o = oracle_gdn_tree(q, k, v, a, be, S0, parent)
-        S = oracle_gdn_commit(k, v, a, be, S0, parent, path, plen)
-        o2, S2 = packed_gdn(q, k, v, a, be, S0, parent, path, plen)
-        np.testing.assert_allclose(o2, o, rtol=1e-10, atol=1e-10)
-        np.testing.assert_allclose(S2, S, rtol=1e-10, atol=1e-10)
+        er = np.random.default_rng(seed + 7).uniform(0.0, 1.0, size=be.shape)
+        for erase in (None, er):
+            o = oracle_gdn_tree(q, k, v, a, be, S0, parent, erase=erase)
+            S = oracle_gdn_commit(k, v, a, be, S0, parent, path, plen, erase=erase)
+            o2, S2 = packed_gdn(q, k, v, a, be, S0, parent, path, plen, erase=erase)
+            np.testing.assert_allclose(o2, o, rtol=1e-10, atol=1e-10)
+            np.testing.assert_allclose(S2, S, rtol=1e-10, atol=1e-10)
 
 
 def test_gdn_pins_catch_planted_mistakes():
     import oracle.gdn as gd
     src = open(gd.__file__).read()
-    step = "    return a * (S - be * np.outer(S @ kj, kj)) + be * np.outer(vj, kj)\n"
+    step = "    return a * (S - er * np.outer(S @ kj, kj)) + be * np.outer(vj, kj)\n"
     assert src.count(step) == 1
     mutants = {
-        "gate after the write": (step, "    return a * (S - be * np.outer(S @ kj, kj) + be * np.outer(vj, kj))\n"),
-        "no beta on the write": (step, "    return a * (S - be * np.outer(S @ kj, kj)) + np.outer(vj, kj)\n"),
+        "gate after the write": (step, "    return a * (S - er * np.outer(S @ kj, kj) + be * np.outer(vj, kj))\n"),
+        "no beta on the write": (step, "    return a * (S - er * np.outer(S @ kj, kj)) + np.outer(vj, kj)\n"),
         "no erase (plain linear attention)": (step, "    return a * S + be * np.outer(vj, kj)\n"),
+        "write strength erases": (step, "    return a * (S - be * np.outer(S @ kj, kj)) + be * np.outer(vj, kj)\n"),
+        "erase strength writes": (step, "    return a * (S - er * np.outer(S @ kj, kj)) + er * np.outer(vj, kj)\n"),
         "heads round robin": ("                g = h // grp\n                S = S0[s, h].copy()\n                for j in path:",
                               "                g = h % Hk\n                S = S0[s, h].copy()\n                for j in path:"),
         "root skipped": ("    return out[::-1]\n", "    return out[::-1][1:]\n"),
     }
     checks = [test_golden_hand_worked_tree, test_beta_zero_is_pure_decay, test_unit_write_maps_the_key_to_its_value,
               test_orthonormal_keys_recall_every_value_on_the_path, test_each_node_equals_its_path_decoded_alone,
-              test_identical_siblings_and_commit_at_the_leaf, test_packed_triangular_solve_equals_the_walk]
+              test_identical_siblings_and_commit_at_the_leaf, test_golden_decoupled_erase_and_write,
+              test_zero_erase_is_gated_linear_attention, test_packed_triangular_solve_equals_the_walk]
     g = globals()
     for name, (old, new) in mutants.items():
         assert src.count(old) >= 1, name
