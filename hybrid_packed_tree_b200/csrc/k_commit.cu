@@ -210,6 +210,94 @@ __global__ void __launch_bounds__(kCThreads, 4) commit_stream_kernel(const Commi
     }
 }
 
+// The same stream for dstate 128 (slabs of 64 rows): thread t owns the four state
+// columns 4 (t % 32) .. +3 of rows t / 32 + 8k, k = 0..7, so each path position
+// costs one shared-memory read of its B columns for all eight rows; the staged x
+// values already carry the position's weight, and the updates go two lanes per
+// fp32x2 FMA.
+__global__ void __launch_bounds__(kCThreads, 4) commit_stream128_kernel(const CommitParams p)
+{
+    constexpr int N = 128, R = 64, kRowsPerThread = R * N / 4 / kCThreads;   // 8
+    __shared__ __align__(16) float Bq[kQChunk * N];          // staged path rows of B
+    __shared__ float cfq[kQChunk * R];                       // w_q x_q[row]
+    __shared__ int32_t pn[kMaxNodes];
+    __shared__ float wq[kMaxNodes];
+    __shared__ int32_t s_len;
+    __shared__ float s_alpha;
+
+    const int tid = threadIdx.x;
+    const int H = p.H, P = p.P, G = p.G, T = p.T;
+    const int chunk = blockIdx.x % p.chunks;
+    const int h = (blockIdx.x / p.chunks) % H;
+    const int b = blockIdx.x / (p.chunks * H);
+    const int g = h / (H / G);
+    const int p0 = chunk * R, rows = min(R, P - p0);
+    const int c4 = tid & 31, r0 = tid >> 5;
+
+    const float4 *src = reinterpret_cast<const float4 *>(p.h0 + (((size_t)b * H + h) * P + p0) * N);
+    float4 hv[kRowsPerThread];
+#pragma unroll
+    for (int k = 0; k < kRowsPerThread; ++k) {
+        hv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r0 + 8 * k < rows)
+            asm volatile("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(hv[k].x), "=f"(hv[k].y), "=f"(hv[k].z), "=f"(hv[k].w)
+                         : "l"(src + tid + k * kCThreads)
+                         : "memory");
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid == 0) {
+        s_len = p.ws.len[b];
+        s_alpha = p.ws.alpha[(size_t)b * H + h];
+    }
+    if (tid < p.Lc) {
+        pn[tid] = p.ws.pn[(size_t)b * p.Lc + tid];
+        wq[tid] = p.ws.w[((size_t)b * H + h) * p.Lc + tid];
+    }
+    __syncthreads();
+    const int len = s_len;
+    if (len < 0) return;                             // invalid tree or path: h_new untouched
+    const float al = s_alpha;
+    float2 acc[kRowsPerThread][2];
+#pragma unroll
+    for (int k = 0; k < kRowsPerThread; ++k) {
+        acc[k][0] = make_float2(al * hv[k].x, al * hv[k].y);
+        acc[k][1] = make_float2(al * hv[k].z, al * hv[k].w);
+    }
+    const size_t xrow = (size_t)H * P;
+    for (int q0 = 0; q0 < len; q0 += kQChunk) {
+        const int nq = min(kQChunk, len - q0);
+        if (q0 > 0) __syncthreads();
+        for (int e = tid; e < nq * N; e += kCThreads) {
+            const int qq = e >> 7;
+            Bq[e] = load_as_float(p.B, (((size_t)b * T + pn[q0 + qq]) * G + g) * N + (e & (N - 1)), p.dtype);
+        }
+        for (int e = tid; e < nq * R; e += kCThreads) {
+            const int qq = e >> 6, r = e & (R - 1);
+            cfq[e] = r < rows ? wq[q0 + qq] * load_as_float(p.x, ((size_t)b * T + pn[q0 + qq]) * xrow +
+                                                                       (size_t)h * P + p0 + r, p.dtype)
+                              : 0.f;
+        }
+        __syncthreads();
+        for (int qq = 0; qq < nq; ++qq) {
+            const float4 bv = *reinterpret_cast<const float4 *>(Bq + qq * N + 4 * c4);
+            const float2 b01 = make_float2(bv.x, bv.y), b23 = make_float2(bv.z, bv.w);
+#pragma unroll
+            for (int k = 0; k < kRowsPerThread; ++k) {
+                const float cf = cfq[qq * R + r0 + 8 * k];
+                const float2 cc = make_float2(cf, cf);
+                acc[k][0] = ptx::ffma2(cc, b01, acc[k][0]);
+                acc[k][1] = ptx::ffma2(cc, b23, acc[k][1]);
+            }
+        }
+    }
+    float4 *dst = reinterpret_cast<float4 *>(p.h_new + (((size_t)b * H + h) * P + p0) * N);
+#pragma unroll
+    for (int k = 0; k < kRowsPerThread; ++k)
+        if (r0 + 8 * k < rows)
+            __stcs(dst + tid + k * kCThreads, make_float4(acc[k][0].x, acc[k][0].y, acc[k][1].x, acc[k][1].y));
+}
+
 }  // namespace
 
 bool commit_supported(const ScanArgs &a)
@@ -261,6 +349,7 @@ cudaError_t launch_commit(const ScanArgs &a, const CommitWork &ws, cudaStream_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (a.N == 128 && p.R == 64) return cudaLaunchKernelEx(&cfg, commit_stream128_kernel, p);
     return cudaLaunchKernelEx(&cfg, commit_stream_kernel, p);
 }
 

@@ -61,6 +61,7 @@ CASES = [
     ("m2_2p7b", None, 384, [383], 32, 4),
     ("hyb8b", 2, 256, [256, 100], 8, 8),
     ("wide256_chain", 1, 256, [200], 16, 16),
+    ("wide256", 2, 512, [512, 300], 32, 8),
     ("hyb8b", 1, 4096, [4096], 32, 8),                 # 33 key blocks over many splits
     ("serve64", 2, 2048, [2047, 129], 64, 8),          # two query tiles per head group
 ]

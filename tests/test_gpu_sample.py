@@ -74,6 +74,8 @@ def test_sampling_golden_cases(st):
 
 CASES = [
     # (workload, batch, vocab, logits dtype, temperature, maxlen or None = n_nodes)
+    ("tiny", None, 64, "f32", 1.0, None),
+    ("tiny", 3, 100, "bf16", 0.9, None),
     ("m2_2p7b", None, 50280, "bf16", 1.0, None),
     ("serve64", 4, 50280, "bf16", 0.7, None),
     ("serve64", 64, 4096, "f32", 1.0, None),
