@@ -5,11 +5,13 @@
 // one triangular solve, and only the accepted state rebuilt on commit from a small
 // pseudo-value matrix instead of per-node states; "Bole" abstract: the
 // tree-structured closed form of the linear-attention recurrence).  Per sequence
-// and value head, with state S [d_v, d_k]:
-//   S_i = alpha_i S_p(i) (I - beta_i k_i k_i^T) + beta_i v_i k_i^T,  S_p(root) = S0,  o_i = S_i q_i.
-// Writing S_t = alpha_t S_{t-1} + u_t k_t^T with u_t = beta_t (v_t - alpha_t S_{t-1} k_t)
+// and value head, with state S [d_v, d_k], write strength beta and erase strength a
+// (a = beta for the gated delta rule; apart, the decoupled erase and write of
+// Gated DeltaNet-2; a = 0, gated linear attention):
+//   S_i = alpha_i S_p(i) (I - a_i k_i k_i^T) + beta_i v_i k_i^T,  S_p(root) = S0,  o_i = S_i q_i.
+// Writing S_t = alpha_t S_{t-1} + u_t k_t^T with u_t = beta_t v_t - a_t alpha_t S_{t-1} k_t
 // and gamma_i for the product of alpha over the root path of i:
-//   u_j   = beta_j (v_j - gamma_j S0 k_j) - sum_{l strict ancestor of j} beta_j (gamma_j / gamma_l) (k_j . k_l) u_l
+//   u_j   = beta_j v_j - a_j gamma_j S0 k_j - sum_{l strict ancestor of j} a_j (gamma_j / gamma_l) (k_j . k_l) u_l
 //   o_i   = gamma_i S0 q_i + sum_{j in anc(i)} (gamma_i / gamma_j) (q_i . k_j) u_j
 //   S_new = gamma_leaf S0 + sum_{j on path} (gamma_leaf / gamma_j) u_j k_j^T
 // The system for u is lower triangular over the ancestor relation: nodes of one
@@ -49,7 +51,7 @@ constexpr int kMaxDevices = 64;
 
 struct GdnParams {
     const void *q, *k, *v;
-    const float *alpha, *beta, *S0;
+    const float *alpha, *beta, *erase, *S0;          // erase NULL: a = beta
     const int32_t *parent, *path, *path_len;
     int maxlen;
     void *o;
@@ -61,7 +63,7 @@ struct GdnParams {
 enum GdnMisc { G_BADI = 0, G_BADQ, G_LEN, G_TREEOK, G_PATHOK, G_COMMIT, G_DATAOK, G_MAXD, kGdnMisc };
 
 struct GdnLayout {
-    uint32_t q, k, v, o, rq, rk, u, mq, ak, lg, eg, be, la, par, dep, anc, praw, pnode, wq, misc, bar, total;
+    uint32_t q, k, v, o, rq, rk, u, mq, ak, lg, eg, be, er, la, par, dep, anc, praw, pnode, wq, misc, bar, total;
     __host__ __device__ GdnLayout(int T, int e)
     {
         uint32_t off = 0;
@@ -82,6 +84,7 @@ struct GdnLayout {
         lg = take((uint32_t)T * 4);
         eg = take((uint32_t)T * 4);
         be = take((uint32_t)T * 4);
+        er = take((uint32_t)T * 4);
         la = take((uint32_t)T * 4);
         par = take((uint32_t)T * 4);
         dep = take((uint32_t)T * 4);
@@ -118,7 +121,8 @@ __global__ void __launch_bounds__(kThreadsG, 2) gdn_tree_kernel(const GdnParams 
     float *Ak = reinterpret_cast<float *>(sm + ly.ak);   // [T][T]   beta_i (gamma_i / gamma_j) k_i . k_j
     float *lg = reinterpret_cast<float *>(sm + ly.lg);   // log gamma
     float *eg = reinterpret_cast<float *>(sm + ly.eg);   // gamma
-    float *bes = reinterpret_cast<float *>(sm + ly.be);  // beta
+    float *bes = reinterpret_cast<float *>(sm + ly.be);  // beta (write)
+    float *ers = reinterpret_cast<float *>(sm + ly.er);  // erase strength
     float *las = reinterpret_cast<float *>(sm + ly.la);  // log alpha
     int32_t *par = reinterpret_cast<int32_t *>(sm + ly.par);
     int32_t *dep = reinterpret_cast<int32_t *>(sm + ly.dep);
@@ -147,13 +151,14 @@ __global__ void __launch_bounds__(kThreadsG, 2) gdn_tree_kernel(const GdnParams 
     // ---------------------------------------------------------------- 1. loads
     const int plim = min(p.maxlen, T);
     int par_v = 0, path_v = 0, len_v = 0;
-    float al_v = 1.f, be_v = 0.f;
+    float al_v = 1.f, be_v = 0.f, er_v = 0.f;
     float4 hv[8];                                         // root warps: rows 8 w + r of S0
     if (tree_warp) {
         if (ttid < T) {
             par_v = p.parent[(size_t)b * T + ttid];
             al_v = p.alpha[((size_t)b * T + ttid) * Hv + h];
             be_v = p.beta[((size_t)b * T + ttid) * Hv + h];
+            er_v = p.erase ? p.erase[((size_t)b * T + ttid) * Hv + h] : be_v;
         }
         if (do_commit && ttid < plim) path_v = p.path[(size_t)b * p.maxlen + ttid];
         if (do_commit && ttid == 0) len_v = p.path_len[b];
@@ -201,6 +206,7 @@ __global__ void __launch_bounds__(kThreadsG, 2) gdn_tree_kernel(const GdnParams 
             par[ttid] = par_v;
             las[ttid] = logf(al_v);
             bes[ttid] = be_v;
+            ers[ttid] = er_v;
         }
         if (do_commit && ttid < plim) praw[ttid] = path_v;
         if (ttid == 0) {
@@ -296,7 +302,7 @@ __global__ void __launch_bounds__(kThreadsG, 2) gdn_tree_kernel(const GdnParams 
                 if (valid && quarter == 0) {
                     const float r = expf(lg[i] - lg[j]);
                     Mq[i * T + j] = r * dq;
-                    if (j != i) Ak[i * T + j] = bes[i] * r * dk;
+                    if (j != i) Ak[i * T + j] = ers[i] * r * dk;
                 }
             }
         }
@@ -345,7 +351,8 @@ __global__ void __launch_bounds__(kThreadsG, 2) gdn_tree_kernel(const GdnParams 
         for (int e = tid; e < T * kRows; e += kThreadsG) {
             const int j = e / kRows, row = e - j * kRows;
             if (dep[j] != d) continue;
-            float u = bes[j] * (in_to_f(vs[e]) - eg[j] * Rk[e]);
+            float u = p.erase ? bes[j] * in_to_f(vs[e]) - ers[j] * eg[j] * Rk[e]
+                              : bes[j] * (in_to_f(vs[e]) - eg[j] * Rk[e]);
             const float *Aj = Ak + j * T;
             for (int wd = 0; wd < 2; ++wd)
                 for (uint32_t bits = ancs[2 * j + wd]; bits; bits &= bits - 1) {
@@ -436,7 +443,8 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 using namespace stree;
 
 extern "C" stree_status stree_gdn_tree_scan_commit(const void *q, const void *k, const void *v, const float *alpha,
-                                                   const float *beta, const float *S0, const int32_t *parent,
+                                                   const float *beta, const float *erase, const float *S0,
+                                                   const int32_t *parent,
                                                    int n_nodes, int batch, int heads_v, int heads_k, int dk, int dv,
                                                    stree_dtype dtype, const int32_t *accepted_path,
                                                    const int32_t *path_len, int maxlen, void *o, float *S_new,
@@ -454,7 +462,7 @@ extern "C" stree_status stree_gdn_tree_scan_commit(const void *q, const void *k,
     for (const void *ptr : ptrs16)
         if (!aligned(ptr, 16)) return STREE_ERR_MISALIGNED;
     if (commit && !aligned(S_new, 16)) return STREE_ERR_MISALIGNED;
-    if (!aligned(alpha, 4) || !aligned(beta, 4) || !aligned(parent, 4) || !aligned(err_out, 4) ||
+    if (!aligned(alpha, 4) || !aligned(beta, 4) || !aligned(erase, 4) || !aligned(parent, 4) || !aligned(err_out, 4) ||
         (commit && (!aligned(accepted_path, 4) || !aligned(path_len, 4))))
         return STREE_ERR_MISALIGNED;
     const long long grid = (long long)batch * heads_v * (dv / kRows);
@@ -464,7 +472,7 @@ extern "C" stree_status stree_gdn_tree_scan_commit(const void *q, const void *k,
     int32_t *err = err_out;
     if (err && cudaMemsetAsync(err, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return STREE_ERR_CUDA;
     GdnParams p{};
-    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.S0 = S0;
+    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.erase = erase; p.S0 = S0;
     p.parent = parent;
     p.path = commit ? accepted_path : nullptr;
     p.path_len = commit ? path_len : nullptr;

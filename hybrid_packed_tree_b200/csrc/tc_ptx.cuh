@@ -42,24 +42,13 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-#ifndef STREE_WAIT_HINT_NS
-#define STREE_WAIT_HINT_NS 20000u
-#endif
-
-// The thread may sleep in the instruction (up to the hint) until the phase
-// completes, so a waiting warp does not take issue slots from working ones.
+// The thread may be suspended in the instruction (for a time the hardware
+// chooses) until the phase completes, so a waiting warp does not take issue slots
+// from working ones.  (An explicit suspend-time hint measured slower: waking
+// later than the phase completion.)
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
-#if STREE_WAIT_HINT_NS > 0
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"((uint32_t)STREE_WAIT_HINT_NS)
-        : "memory");
-#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -67,7 +56,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
-#endif
     return ok != 0;
 }
 

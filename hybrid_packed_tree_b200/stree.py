@@ -63,7 +63,7 @@ _lib.stree_unrolled_scan.argtypes = [_vp] * 9 + [_i] * 9 + [_vp, _vp, _vp, _vp]
 _lib.stree_accept_greedy.argtypes = [_vp, _i, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.stree_accept_sampling.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _i, _i, ctypes.c_float, _vp, _vp, _i, _vp,
                                         _vp, _vp, _vp, _vp]
-_lib.stree_gdn_tree_scan_commit.argtypes = [_vp] * 7 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp, _vp]
+_lib.stree_gdn_tree_scan_commit.argtypes = [_vp] * 8 + [_i] * 7 + [_vp, _vp, _i, _vp, _vp, _vp, _vp]
 _lib.stree_tree_attention.argtypes = [_vp] * 7 + [_i] * 6 + [ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp, _vp]
 _lib.stree_tree_attention_workspace_size.argtypes = [_i] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
 _lib.stree_sync_check.argtypes = [_vp, _vp, _ip]
@@ -310,18 +310,19 @@ def stree_accept_sampling(target_logits, draft_logits, draft_tokens, parent, tem
 
 
 def stree_gdn_tree_scan_commit(q, k, v, alpha, beta, S0, parent, o, path=None, path_len=None, S_new=None,
-                               err_out=None, stream=None):
+                               err_out=None, stream=None, erase=None):
     """Gated delta rule over the packed tree: o [b, T, Hv, dv] for every node and, when
     path / path_len / S_new are given, the accepted path's state S_new [b, Hv, dv, dk].
     q, k [b, T, Hk, dk] and v [b, T, Hv, dv] in one dtype (fp32 or bf16); alpha, beta
-    [b, T, Hv] and S0 fp32."""
+    [b, T, Hv] and S0 fp32; erase [b, T, Hv] fp32 (None: erase = beta; zeros: gated
+    linear attention)."""
     batch, T, Hk, dk = k.shape
     Hv, dv = v.shape[2], v.shape[3]
     io = (v.dtype,)
     st = _lib.stree_gdn_tree_scan_commit(
         _ptr(q, "q", io), _ptr(k, "k", io), _ptr(v, "v", (torch.float32, torch.bfloat16)),
         _ptr(alpha, "alpha", (torch.float32,)), _ptr(beta, "beta", (torch.float32,)),
-        _ptr(S0, "S0", (torch.float32,)), _ptr(parent, "parent", (torch.int32,)), T, batch, Hv, Hk, dk, dv,
+        _ptr(erase, "erase", (torch.float32,)), _ptr(S0, "S0", (torch.float32,)), _ptr(parent, "parent", (torch.int32,)), T, batch, Hv, Hk, dk, dv,
         _io_dtype(v), _ptr(path, "path", (torch.int32,)), _ptr(path_len, "path_len", (torch.int32,)),
         path.shape[1] if path is not None else 0, _ptr(o, "o", io), _ptr(S_new, "S_new", (torch.float32,)),
         _ptr(err_out, "err_out", (torch.int32,)), _stream(stream))

@@ -307,18 +307,23 @@ stree_status stree_accept_sampling(const void *target_logits, const void *draft_
  * draft node's output from one triangular solve and only the accepted state
  * rebuilt on commit; "Bole" abstract: the tree-structured closed form of the
  * linear-attention recurrence).  Per sequence and value head h (query/key head
- * g = h / (heads_v / heads_k)), node i with parent p(i):
- *     S_i = alpha_i S_p(i) (I - beta_i k_i k_i^T) + beta_i v_i k_i^T,  S_p(root) = S0[b,h]
+ * g = h / (heads_v / heads_k)), node i with parent p(i), write strength beta and
+ * erase strength a:
+ *     S_i = alpha_i S_p(i) (I - a_i k_i k_i^T) + beta_i v_i k_i^T,  S_p(root) = S0[b,h]
  *     o_i = S_i q_i
- * computed through the pseudo-values u (an ancestor-triangular solve) and
+ * With erase NULL, a = beta: the gated delta rule.  Given apart, the decoupled
+ * erase and write of Gated DeltaNet-2 (related entry on the TreeWY page); all
+ * zero, gated linear attention (S_i = alpha_i S_p(i) + beta_i v_i k_i^T).
+ * Computed through the pseudo-values u (an ancestor-triangular solve) and
  * gamma_i = product of alpha over the root path of i:
- *     u_j   = beta_j (v_j - gamma_j S0 k_j) - sum_{l strict ancestor of j} beta_j (gamma_j/gamma_l) (k_j . k_l) u_l
+ *     u_j   = beta_j v_j - a_j gamma_j S0 k_j - sum_{l strict ancestor of j} a_j (gamma_j/gamma_l) (k_j . k_l) u_l
  *     o_i   = gamma_i S0 q_i + sum_{j in anc(i)} (gamma_i/gamma_j) (q_i . k_j) u_j
  *     S_new = gamma_leaf S0 + sum_{j on path} (gamma_leaf/gamma_j) u_j k_j^T   (S0 for an empty path)
  *
  *   q, k   [batch, n_nodes, heads_k, dk]   dtype (fp32 or bf16)
  *   v, o   [batch, n_nodes, heads_v, dv]   dtype
  *   alpha, beta [batch, n_nodes, heads_v]  fp32 (gate in (0, 1] and write strength, after activation)
+ *   erase       [batch, n_nodes, heads_v]  fp32 erase strength, or NULL (erase = beta)
  *   S0, S_new   [batch, heads_v, dv, dk]   fp32 (S_new may alias S0)
  *   parent [batch, n_nodes], accepted_path [batch, maxlen], path_len [batch] int32: as for the scan
  *   err_out device int32[4] error word of this call (cleared by the call), or NULL
@@ -331,7 +336,8 @@ stree_status stree_accept_sampling(const void *target_logits, const void *draft_
  * owns every buffer; the call allocates nothing and runs on `stream`.
  */
 stree_status stree_gdn_tree_scan_commit(const void *q, const void *k, const void *v, const float *alpha,
-                                        const float *beta, const float *S0, const int32_t *parent, int n_nodes,
+                                        const float *beta, const float *erase, const float *S0,
+                                        const int32_t *parent, int n_nodes,
                                         int batch, int heads_v, int heads_k, int dk, int dv, stree_dtype dtype,
                                         const int32_t *accepted_path, const int32_t *path_len, int maxlen, void *o,
                                         float *S_new, int32_t *err_out, void *stream);

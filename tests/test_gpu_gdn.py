@@ -2,7 +2,8 @@
 the fp64 oracle: every node's output and the committed state, element by element,
 at the tolerances of the scan (1e-4 max|ref| for fp32 inputs, 2e-2 for bf16);
 invalid trees and paths, the empty path, the in-place commit and the call
-without a commit."""
+without a commit; the erase strength apart from the write strength (random, and
+zero: gated linear attention)."""
 import numpy as np
 import pytest
 import torch
@@ -30,22 +31,24 @@ def _upload(g):
     return d
 
 
-def _run(st, g, d, commit=True, S_new=None):
+def _run(st, g, d, commit=True, S_new=None, erase=None):
     o = torch.full_like(d["v"], 7.0)
     if commit and S_new is None:
         S_new = torch.full_like(d["S0"], 7.0)
     err = torch.full((4,), -1, dtype=torch.int32, device="cuda")
     st.stree_gdn_tree_scan_commit(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], d["parent"], o,
                                   d["path"] if commit else None, d["path_len"] if commit else None,
-                                  S_new if commit else None, err_out=err)
+                                  S_new if commit else None, err_out=err,
+                                  erase=None if erase is None else to_dev(erase, "f32"))
     torch.cuda.synchronize()
     return o, S_new, err.tolist()
 
 
-def _oracle(g):
+def _oracle(g, erase=None):
     f = g.f64()
-    o = oracle_gdn_tree(f["q"], f["k"], f["v"], f["alpha"], f["beta"], f["S0"], g.parent)
-    S = oracle_gdn_commit(f["k"], f["v"], f["alpha"], f["beta"], f["S0"], g.parent, g.path, g.path_len)
+    o = oracle_gdn_tree(f["q"], f["k"], f["v"], f["alpha"], f["beta"], f["S0"], g.parent, erase=erase)
+    S = oracle_gdn_commit(f["k"], f["v"], f["alpha"], f["beta"], f["S0"], g.parent, g.path, g.path_len,
+                          erase=erase)
     return o, S
 
 
@@ -69,6 +72,25 @@ def test_gdn_matches_oracle(st, name, batch, hv, hk, dv, dtype):
     o_ref, S_ref = _oracle(g)
     assert_close(f64(o), o_ref, dtype, f"{name} o")
     assert_close(f64(S_new), S_ref, dtype, f"{name} S_new")
+
+
+@pytest.mark.parametrize("name,batch,hv,hk,dv,dtype,kind", [
+    ("serve64", 3, 4, 2, 64, "f32", "random"),
+    ("hyb8b", None, 8, 2, 128, "bf16", "random"),
+    ("m2_2p7b", None, 4, 4, 128, "f32", "zero"),
+    ("serve64", 2, 8, 4, 96, "bf16", "zero"),
+])
+def test_gdn_decoupled_erase_matches_oracle(st, name, batch, hv, hk, dv, dtype, kind):
+    w = wl.make_workload(name, batch=batch, layers=1)
+    g = wl.gdn_inputs(w.parent, w.path, w.path_len, heads_v=hv, heads_k=hk, dv=dv, dtype=dtype, seed=43)
+    er = (np.random.default_rng(44).uniform(0.0, 1.0, size=g.beta.shape) if kind == "random"
+          else np.zeros(g.beta.shape)).astype(np.float32)
+    d = _upload(g)
+    o, S_new, err = _run(st, g, d, erase=er)
+    assert err == [0, 0, 0, 0]
+    o_ref, S_ref = _oracle(g, erase=er.astype(np.float64))
+    assert_close(f64(o), o_ref, dtype, f"{name} o ({kind} erase)")
+    assert_close(f64(S_new), S_ref, dtype, f"{name} S_new ({kind} erase)")
 
 
 def test_gdn_chain_of_64_and_empty_path_in_place(st):
