@@ -293,8 +293,8 @@ __global__ void __launch_bounds__(kThreadsG, 2) gdn_tree_kernel(const GdnParams 
                     if (a0) a0 &= a0 - 1; else a1 &= a1 - 1;
                 }
                 const int j = valid ? (a0 ? __ffs(a0) - 1 : 32 + __ffs(a1) - 1) : i;
-                float dq = dot32(qs, ks, i, j, quarter);
-                float dk = dot32(ks, ks, i, j, quarter);
+                float dq = dot32(qs, ks, i, j, quarter, dot32_rot<In>(lane));
+                float dk = dot32(ks, ks, i, j, quarter, dot32_rot<In>(lane));
                 dq += __shfl_xor_sync(0xffffffffu, dq, 1);
                 dk += __shfl_xor_sync(0xffffffffu, dk, 1);
                 dq += __shfl_xor_sync(0xffffffffu, dq, 2);

@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kThreadsS, 2) scan_small_kernel(const SmallPar
                     if (a0) a0 &= a0 - 1; else a1 &= a1 - 1;
                 }
                 const int j = valid ? (a0 ? __ffs(a0) - 1 : 32 + __ffs(a1) - 1) : i;
-                float d = dot32(Cs, Bs, i, j, quarter);
+                float d = dot32(Cs, Bs, i, j, quarter, dot32_rot<In>(lane));
                 d += __shfl_xor_sync(0xffffffffu, d, 1);
                 d += __shfl_xor_sync(0xffffffffu, d, 2);
                 if (valid && quarter == 0) Ms[i * T + j] = expf(Ls[i] - Ls[j]) * d * dts[j] + (i == j ? Dh : 0.f);

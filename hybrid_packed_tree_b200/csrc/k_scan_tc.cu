@@ -151,32 +151,30 @@ __device__ __forceinline__ float dot_cb(const uint8_t *cs, int T_pad, const __nv
     return acc;
 }
 
-// C_i . B_j over the quarter `part` (32 of the 128 state columns); four lanes of
-// a warp combine their parts with shuffles.  B_j is read from shared memory
-// (kStaged) or from global memory.  The eight pairs of a warp walk their 4-column
-// chunks in rotated order (`rot`): B rows lie 256 bytes apart, so the same chunk
-// of different rows would fall into the same shared-memory banks.
+// C_i . B_j over all 128 state columns by one lane.  The lane walks the 32
+// four-column chunks starting at chunk `rot` (its lane index), so the lanes of a
+// warp read 32 different chunks of their B rows (rows lie 256 bytes apart,
+// unswizzled: without the rotation they would all hit the same banks) and spread
+// their C reads over the swizzle's eight 16-byte bank groups.  Four accumulators,
+// one per column of the chunk.
 template <bool kStaged>
-__device__ __forceinline__ float dot_cb_part(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i, int part,
-                                             int rot)
+__device__ __forceinline__ float dot_cb_lane(const uint8_t *cs, int T_pad, const __nv_bfloat16 *Bj, int i, int rot)
 {
-    float acc = 0.f;
-    const uint8_t *crow = cs + part * T_pad * 128 + i * 128;     // K-atom `part` holds columns 32*part..
-    const uint2 *brow = reinterpret_cast<const uint2 *>(Bj) + part * 8;
-    uint2 raw[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) raw[c] = kStaged ? brow[(c + rot) & 7] : __ldg(brow + ((c + rot) & 7));
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const float4 cv = *reinterpret_cast<const float4 *>(crow + ((((c + rot) & 7) ^ (i & 7)) << 4));
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    const uint2 *brow = reinterpret_cast<const uint2 *>(Bj);
+    const uint8_t *crow = cs + i * 128;
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {
+        const int g = (c + rot) & 31;
+        const float4 cv = *reinterpret_cast<const float4 *>(crow + (g >> 3) * T_pad * 128 + (((g & 7) ^ (i & 7)) << 4));
         float b0, b1, b2, b3;
-        unpack4(raw[c], b0, b1, b2, b3);
-        acc = fmaf(cv.x, b0, acc);
-        acc = fmaf(cv.y, b1, acc);
-        acc = fmaf(cv.z, b2, acc);
-        acc = fmaf(cv.w, b3, acc);
+        unpack4(kStaged ? brow[g] : __ldg(brow + g), b0, b1, b2, b3);
+        a0 = fmaf(cv.x, b0, a0);
+        a1 = fmaf(cv.y, b1, a1);
+        a2 = fmaf(cv.z, b2, a2);
+        a3 = fmaf(cv.w, b3, a3);
     }
-    return acc;
+    return (a0 + a1) + (a2 + a3);
 }
 
 // Byte offset of bf16 element (row, k) in a K-major 128-byte swizzled operand of
@@ -734,17 +732,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                 }
                 __syncthreads();
-                // Four lanes per pair, a quarter of the state columns each.
-                const int part = lane & 3;
-                for (int q0 = (tid >> 2); q0 < ((total + 7) & ~7); q0 += kThreads / 4) {
-                    const int q = q0 < total ? q0 : total - 1;
+                // One lane per pair.
+                for (int q = tid; q < total; q += kThreads) {
                     const int i = pi[q], j = pj[q];
-                    const int rot = (lane >> 2) & 7;
-                    float v = b_staged ? dot_cb_part<true>(cs, T_pad, Bs + j * kDstate, i, part, rot)
-                                       : dot_cb_part<false>(cs, T_pad, Bseq + (size_t)j * brow, i, part, rot);
-                    v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    v += __shfl_xor_sync(0xffffffffu, v, 2);
-                    if (part == 0 && q0 < total) pcb[q] = v;
+                    pcb[q] = b_staged ? dot_cb_lane<true>(cs, T_pad, Bs + j * kDstate, i, lane)
+                                      : dot_cb_lane<false>(cs, T_pad, Bseq + (size_t)j * brow, i, lane);
                 }
             } else if (misc[M_INSMEM] == 2 || p.pcb_g) {
                 // Too many pairs for the fp32 table (deep trees): the products rounded
@@ -753,20 +745,13 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 const bool h16 = misc[M_INSMEM] == 2;
                 const int total = h16 ? (int)misc[M_TOTAL] : min((int)misc[M_TOTAL], p.pair_max);
                 float *pg = h16 ? nullptr : p.pcb_g + (size_t)blockIdx.x * p.pair_max;
-                const int part = lane & 3;
-                for (int q0 = (tid >> 2); q0 < ((total + 7) & ~7); q0 += kThreads / 4) {
-                    const int q = q0 < total ? q0 : total - 1;
+                for (int q = tid; q < total; q += kThreads) {
                     const int i = pair_row(poff, T, q);
                     const int j = nth_set_bit(ancs + i * W, W, q - poff[i]);
-                    const int rot = (lane >> 2) & 7;
-                    float v = b_staged ? dot_cb_part<true>(cs, T_pad, Bs + j * kDstate, i, part, rot)
-                                       : dot_cb_part<false>(cs, T_pad, Bseq + (size_t)j * brow, i, part, rot);
-                    v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    v += __shfl_xor_sync(0xffffffffu, v, 2);
-                    if (part == 0 && q0 < total) {
-                        if (h16) pcb16[q] = __float2bfloat16_rn(v);
-                        else pg[q] = v;
-                    }
+                    const float v = b_staged ? dot_cb_lane<true>(cs, T_pad, Bs + j * kDstate, i, lane)
+                                             : dot_cb_lane<false>(cs, T_pad, Bseq + (size_t)j * brow, i, lane);
+                    if (h16) pcb16[q] = __float2bfloat16_rn(v);
+                    else pg[q] = v;
                 }
             }
             if (p.bs_mh) {                                     // B rows read: clear the region for M_h

@@ -31,24 +31,26 @@ __device__ __forceinline__ float4 row4(const __nv_bfloat16 *base, int row, int l
 }
 
 // C_i . B_j over the 32 state columns 32 s .. 32 s + 31 (four independent sums).
-__device__ __forceinline__ float dot32(const float *C, const float *B, int i, int j, int s)
+__device__ __forceinline__ float dot32(const float *C, const float *B, int i, int j, int s, int rot)
 {
     float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const float4 cv = *reinterpret_cast<const float4 *>(C + i * kCols + 32 * s + 4 * c);
-        const float4 bv = *reinterpret_cast<const float4 *>(B + j * kCols + 32 * s + 4 * c);
+        const int cc = (c + rot) & 7;
+        const float4 cv = *reinterpret_cast<const float4 *>(C + i * kCols + 32 * s + 4 * cc);
+        const float4 bv = *reinterpret_cast<const float4 *>(B + j * kCols + 32 * s + 4 * cc);
         d[c & 3] = fmaf(cv.x, bv.x, fmaf(cv.y, bv.y, fmaf(cv.z, bv.z, fmaf(cv.w, bv.w, d[c & 3]))));
     }
     return (d[0] + d[1]) + (d[2] + d[3]);
 }
-__device__ __forceinline__ float dot32(const __nv_bfloat16 *C, const __nv_bfloat16 *B, int i, int j, int s)
+__device__ __forceinline__ float dot32(const __nv_bfloat16 *C, const __nv_bfloat16 *B, int i, int j, int s, int rot)
 {
     float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        const uint4 cr = *reinterpret_cast<const uint4 *>(C + i * kCols + 32 * s + 8 * c);
-        const uint4 br = *reinterpret_cast<const uint4 *>(B + j * kCols + 32 * s + 8 * c);
+        const int cc = (c + rot) & 3;
+        const uint4 cr = *reinterpret_cast<const uint4 *>(C + i * kCols + 32 * s + 8 * cc);
+        const uint4 br = *reinterpret_cast<const uint4 *>(B + j * kCols + 32 * s + 8 * cc);
         const __nv_bfloat162 *c2 = reinterpret_cast<const __nv_bfloat162 *>(&cr);
         const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&br);
 #pragma unroll
@@ -58,6 +60,17 @@ __device__ __forceinline__ float dot32(const __nv_bfloat16 *C, const __nv_bfloat
         }
     }
     return (d[0] + d[1]) + (d[2] + d[3]);
+}
+
+// Chunk rotation of dot32 for a lane whose pair is lane / 4 and quarter lane % 4.
+// Rows lie 256 (bf16) or 512 (fp32) bytes apart, so without it the lanes of one
+// 16-byte load phase (eight lanes: two pairs, four quarters) would hit the same
+// banks; with it those eight lanes read eight different bank groups.
+template <typename In>
+__device__ __forceinline__ int dot32_rot(int lane)
+{
+    const int pair = (lane >> 2) & 1, quarter = lane & 3;
+    return sizeof(In) == 4 ? 4 * pair + quarter : 2 * pair + (quarter >> 1);
 }
 
 __device__ __forceinline__ void named_sync(int id, int nthreads)
