@@ -63,6 +63,9 @@ def parse():
                     help="skip the unrolled-tree baseline comparison (one layer per workload)")
     ap.add_argument("--no-accept", action="store_true",
                     help="skip the greedy tree-verification timing (argmax over the logits + walk)")
+    ap.add_argument("--no-floor", action="store_true", help="skip the launch and state-copy latency floors")
+    ap.add_argument("--no-attention", action="store_true",
+                    help="skip the tree-masked attention timing (the hybrid's Transformer layers)")
     ap.add_argument("--no-gdn", action="store_true",
                     help="skip the gated-delta-rule tree timing (linear-attention layers)")
     ap.add_argument("--vocab", type=int, default=50280,
@@ -350,11 +353,12 @@ def gdn_bytes(b, T, Hv, Hk, dk, dv, e, maxlen, nodes_on_paths):
             + b * T * 4 + b * maxlen * 4 + b * 4)
 
 
-def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16):
+def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16, linear=False):
     """The gated delta rule over a workload's trees (one linear-attention layer:
     32 value heads, 16 query/key heads, d_k = d_v = 128, bf16 inputs, fp32 state),
     fused with the commit of the workload's accepted paths; a CUDA graph of `steps`
-    calls over rotated buffers after an L2 flush."""
+    calls over rotated buffers after an L2 flush.  linear=True: zero erase strength
+    (gated linear attention; the erase array adds its bytes)."""
     import torch
 
     from hybrid_packed_tree_b200 import stree
@@ -365,6 +369,8 @@ def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16):
     g = wl.gdn_inputs(w.parent, w.path, w.path_len, heads_v=heads_v, heads_k=heads_k, dtype="bf16", seed=41)
     b, T = w.parent.shape
     nbytes = gdn_bytes(b, T, heads_v, heads_k, 128, 128, 2, w.maxlen, int(np.sum(w.path_len)))
+    if linear:
+        nbytes += b * T * heads_v * 4
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     nsets = max(1, -(-3 * l2 // nbytes))
     sets = []
@@ -375,6 +381,7 @@ def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16):
                   for k in ("parent", "path", "path_len")})
         d["o"] = torch.empty_like(d["v"])
         d["S_new"] = torch.empty_like(d["S0"])
+        d["erase"] = torch.zeros_like(d["beta"]) if linear else None
         sets.append(d)
     err = torch.zeros(4, dtype=torch.int32, device=device)
 
@@ -382,7 +389,7 @@ def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16):
         d = sets[i % nsets]
         stree.stree_gdn_tree_scan_commit(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], d["parent"],
                                          d["o"], d["path"], d["path_len"], d["S_new"], err_out=err,
-                                         stream=torch.cuda.current_stream(device))
+                                         stream=torch.cuda.current_stream(device), erase=d["erase"])
 
     for i in range(3):
         call(i)
@@ -406,7 +413,8 @@ def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16):
     del gr
     hbm_gbs, peak_kind = peaks()
     gbs = nbytes / (ms / 1e3) / 1e9
-    return {"workload": f"{name} trees, gated delta rule ({heads_v} value / {heads_k} key heads, d_k = d_v = 128)",
+    rule = "gated linear attention (zero erase)" if linear else "gated delta rule"
+    return {"workload": f"{name} trees, {rule} ({heads_v} value / {heads_k} key heads, d_k = d_v = 128)",
             "batch": b, "n_nodes": T, "ms_per_call": ms, "nodes_per_s": b * T / (ms / 1e3),
             "bytes_per_call": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs,
             "peak_source": f"{peak_kind} hbm_gbs", "kernel": "gdn_tree_kernel",
@@ -480,6 +488,141 @@ def run_sampling(name, vocab, local_rank, steps=20, temperature=1.0):
             "ms_per_call": ms, "accepted_nodes": visited, "bytes_per_call": nbytes, "achieved_gbs": gbs,
             "frac": gbs / hbm_gbs, "peak_source": f"{peak_kind} hbm_gbs",
             "timing": f"{steps} calls in one CUDA graph after an L2 flush, {nsets} rotated copies of the logits"}
+
+
+def run_floor(name, local_rank, steps=200):
+    """Latency floors of one step on this GPU, for comparison with the scan's step
+    time: a CUDA graph of `steps` launches of a one-element kernel (launch and
+    completion only), and of copies of the workload's state (h0 -> h_new, the
+    dominant bytes of the fused step) over rotated buffers after an L2 flush."""
+    import torch
+
+    from hybrid_packed_tree_b200 import workloads as wl
+
+    device = torch.device("cuda", local_rank)
+    w = wl.make_workload(name, layers=1)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    state = w.batch * w.nheads * w.headdim * w.dstate
+    nsets = max(1, -(-3 * l2 // (8 * state)))
+    src = [torch.randn(state, device=device) for _ in range(nsets)]
+    dst = [torch.empty_like(x) for x in src]
+    one = torch.zeros(1, device=device)
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                fn(i)
+        g.replay()
+        flush = torch.empty(int(3 * l2) // 4 + 1, dtype=torch.float32, device=device)
+        flush.zero_()
+        torch.cuda.synchronize(device)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        g.replay()
+        t1.record()
+        torch.cuda.synchronize(device)
+        del g
+        return t0.elapsed_time(t1) / steps * 1e3
+
+    empty_us = timed(lambda i: one.add_(1.0))
+    copy_us = timed(lambda i: dst[i % nsets].copy_(src[i % nsets]))
+    return {"workload": name, "empty_kernel_us": empty_us, "state_copy_us": copy_us,
+            "state_copy_bytes": 8 * state,
+            "note": "CUDA graphs of back-to-back launches: a one-element torch kernel, and a torch copy of the "
+                    "workload's fp32 state (read + write) over rotated buffers"}
+
+
+ATTN_CTX = {"hyb8b": 4096, "serve64": 1024}
+
+
+def run_attention(name, local_rank, steps=20, heads_q=32, heads_kv=8):
+    """Tree-masked attention over a workload's trees (one attention layer of a
+    hybrid model: 32 query heads, 8 key/value heads, head dim 128, bf16), every
+    sequence with a full context of ATTN_CTX[name] cached tokens; a CUDA graph of
+    `steps` calls over rotated buffers after an L2 flush.  Reports HBM bytes (the
+    context keys and values, the tree's, q and o) and the tensor flops actually
+    issued (two 128-row products per key block and query tile)."""
+    import torch
+
+    from hybrid_packed_tree_b200 import stree
+    from hybrid_packed_tree_b200 import workloads as wl
+
+    device = torch.device("cuda", local_rank)
+    w = wl.make_workload(name, layers=1)
+    b, T = w.parent.shape
+    S = ATTN_CTX.get(name, 2048)
+    a = wl.attention_inputs(w.parent, S, [S] * b, heads_q=heads_q, heads_kv=heads_kv, seed=71, stale=0.0)
+    d = 128
+    nbytes = 2 * b * S * heads_kv * d * 2 + 2 * b * T * heads_kv * d * 2 + 2 * b * T * heads_q * d * 2 + b * T * 4
+    G = heads_q // heads_kv
+    tq = 128 // G
+    tiles = b * heads_kv * (-(-T // tq))
+    flops = tiles * 4 * 128 * 128 * d * (-(-S // 128) + 1)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nsets = max(1, -(-3 * l2 // nbytes))
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    base = {k: bf(a[k]) for k in ("q", "k_ctx", "v_ctx", "k_tree", "v_tree")}
+    sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(nsets - 1)]
+    ctx_len = torch.from_numpy(a["ctx_len"]).to(device)
+    parent = torch.from_numpy(a["parent"]).to(device)
+    outs = [torch.empty_like(base["q"]) for _ in range(nsets)]
+    err = torch.zeros(4, dtype=torch.int32, device=device)
+    ws_bytes = stree.stree_tree_attention_workspace_size(T, b, S, heads_q, heads_kv, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device) if ws_bytes else None
+
+    def call(i):
+        t = sets[i % nsets]
+        stree.stree_tree_attention(t["q"], t["k_ctx"], t["v_ctx"], t["k_tree"], t["v_tree"], ctx_len, parent,
+                                   outs[i % nsets], a["scale"], err, workspace=ws,
+                                   stream=torch.cuda.current_stream(device))
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            call(i)
+    g.replay()
+    flush = torch.empty(int(3 * l2) // 4 + 1, dtype=torch.float32, device=device)
+    flush.zero_()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    g.replay()
+    t1.record()
+    torch.cuda.synchronize(device)
+    if int(err[0]) != 0:
+        raise RuntimeError(f"device error in the tree attention: {err.tolist()}")
+    ms = t0.elapsed_time(t1) / steps
+    del g
+    hbm_gbs, peak_kind = peaks()
+    tflops_peak = measured_tflops()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    tfs = flops / (ms / 1e3) / 1e12
+    return {"workload": f"{name} trees, {S} cached tokens per sequence", "batch": b, "n_nodes": T,
+            "heads_q": heads_q, "heads_kv": heads_kv, "head_dim": d, "ms_per_call": ms,
+            "bytes_per_call": nbytes, "achieved_gbs": gbs, "frac_hbm": gbs / hbm_gbs,
+            "tensor_flops_per_call": flops, "achieved_tflops": tfs,
+            "frac_tensor": tfs / tflops_peak if tflops_peak else None, "kernel": "tree_attention_kernel",
+            "workspace_bytes": ws_bytes,
+            "peak_source": f"{peak_kind} hbm_gbs, measured bf16_tflops",
+            "timing": f"{steps} calls in one CUDA graph after an L2 flush, {nsets} rotated buffer sets"}
+
+
+def measured_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def unrolled_summary(o, u):
@@ -706,7 +849,9 @@ def run_separate(torch, stree, w, ctx, sets, nsets, K, device, flush):
     return {
         "scan": {"kernel": KERNEL_NAMES.get(kernel_used, kernel_used), "ms_per_launch": scan_ms,
                  "bytes_per_launch": scan_bytes(w)},
-        "commit": {"kernel": "commit_kernel", "ms_per_launch": commit_ms, "bytes_per_launch": commit_bytes(w)},
+        "commit": {"kernel": "commit_prep_kernel + " + ("commit_stream128_kernel" if w.dstate == 128 and w.headdim >= 64
+                                                         else "commit_stream_kernel"),
+                   "ms_per_launch": commit_ms, "bytes_per_launch": commit_bytes(w)},
         "timing": f"{K} steps x {nl} layers of scan-then-commit in one CUDA graph after an L2 flush, "
                   "timing events around every call",
     }
@@ -877,6 +1022,9 @@ def main():
                 out["other_workloads"][name]["accept_sampling"] = run_sampling(name, args.vocab, local_rank)
             if not args.no_gdn and rank == 0 and name in SIDE_WORKLOADS:
                 out["other_workloads"][name]["gdn_tree"] = run_gdn(name, local_rank)
+                out["other_workloads"][name]["gla_tree"] = run_gdn(name, local_rank, linear=True)
+            if not args.no_attention and rank == 0 and name in ATTN_CTX:
+                out["other_workloads"][name]["tree_attention"] = run_attention(name, local_rank)
     if rank == 0 and not args.no_unrolled:
         out["unrolled_baseline"] = unrolled_summary(out, run_unrolled(args.config, local_rank))
     if rank == 0 and not args.no_accept:
@@ -884,6 +1032,11 @@ def main():
         out["accept_sampling"] = run_sampling(args.config, args.vocab, local_rank)
     if rank == 0 and not args.no_gdn:
         out["gdn_tree"] = run_gdn(args.config, local_rank)
+        out["gla_tree"] = run_gdn(args.config, local_rank, linear=True)
+    if rank == 0 and not args.no_attention and args.config in ATTN_CTX:
+        out["tree_attention"] = run_attention(args.config, local_rank)
+    if rank == 0 and not args.no_floor:
+        out["latency_floor"] = run_floor(args.config, local_rank)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(args.config, args.cpu_seconds)
     if rank == 0:

@@ -553,33 +553,20 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 const int q = tid + u * kThreads, hh = q / T, i = q - hh * T;
                 if (q < hpt * T) dtv[u] = p.dt[((size_t)b * T + i) * H + hfirst + hh];
             }
-            {
-                // All of this thread's C loads are issued before the first is used.
-                constexpr int kCItems = (kMaxTcNodes * 32 + kThreads - 1) / kThreads;
-                uint2 raw[kCItems];
+            // All of this thread's C loads are issued here and first used after the
+            // tree is rebuilt, so their latency overlaps that work.
+            constexpr int kCItems = (kMaxTcNodes * 32 + kThreads - 1) / kThreads;
+            uint2 craw[kCItems];
 #pragma unroll
-                for (int u = 0; u < kCItems; ++u) {
-                    const int q = tid + u * kThreads, i = q >> 5, c = q & 31;
-                    raw[u] = make_uint2(0u, 0u);
-                    if (i < T)
-                        raw[u] = __ldg(reinterpret_cast<const uint2 *>(p.C + (((size_t)b * T + i) * G + g) * kDstate + c * 4));
-                }
-#pragma unroll
-                for (int u = 0; u < kCItems; ++u) {
-                    const int q = tid + u * kThreads, i = q >> 5, c = q & 31;
-                    if (q < T_pad * 32) {
-                        float4 v;
-                        unpack4(raw[u], v.x, v.y, v.z, v.w);
-                        *reinterpret_cast<float4 *>(cs + (c >> 3) * T_pad * 128 + i * 128 + (((c & 7) ^ (i & 7)) << 4)) = v;
-                    }
-                }
+            for (int u = 0; u < kCItems; ++u) {
+                const int q = tid + u * kThreads, i = q >> 5, c = q & 31;
+                craw[u] = make_uint2(0u, 0u);
+                if (i < T)
+                    craw[u] = __ldg(reinterpret_cast<const uint2 *>(p.C + (((size_t)b * T + i) * G + g) * kDstate + c * 4));
             }
             if (new_b && !p.bs_mh)
                 for (uint32_t o = tid * 16u; o < (uint32_t)hpt * p.mh_head; o += kThreads * 16u)
                     *reinterpret_cast<float4 *>(mh + o) = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-                if (tid + u * kThreads < hpt * T) coef(k & 1, 0)[tid + u * kThreads] = bf2f(dtv[u]);
             if (tid == 0) {
                 misc[M_DTK] = (int)k + 1;
                 if (new_b) {
@@ -595,9 +582,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 if (p.parent) {
                     // Phase 2a: the tree itself -- node 0 the only root, every other
                     // parent an earlier node -- then each node's ancestor-or-self row
-                    // and depth by walking its root path.  An invalid tree is reported
-                    // by the tree builder launched with this kernel; here its tiles
-                    // flow through the pipeline with empty masks and are not stored.
+                    // (built in registers) and depth by walking its root path.  An
+                    // invalid tree is reported by the CTA holding the sequence's first
+                    // tile; its tiles flow through the pipeline with empty masks and
+                    // are not stored.
                     int bad = 0;
                     for (int i = tid; i < T; i += kThreads) {
                         const int v = par[i];
@@ -605,13 +593,18 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                     }
                     okb = !__syncthreads_or(bad);
                     for (int i = tid; i < T; i += kThreads) {
-                        for (int w = 0; w < W; ++w) ancs[i * W + w] = 0u;
+                        uint32_t a4[4] = {0u, 0u, 0u, 0u};                // W <= 4 (T <= 128)
                         int d = -1;
                         if (okb)
                             for (int j = i; j >= 0; j = par[j]) {
-                                ancs[i * W + (j >> 5)] |= 1u << (j & 31);
+                                const uint32_t bit = 1u << (j & 31), wq = (uint32_t)j >> 5;
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) a4[u] |= wq == (uint32_t)u ? bit : 0u;
                                 ++d;
                             }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (u < W) ancs[i * W + u] = a4[u];
                         dep[i] = okb ? d : 0;
                     }
                     if (tid == 0) misc[M_OK] = okb;
@@ -688,6 +681,19 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_h0, const __grid_constant_
                 }
                 cur_b = b;
             }
+            // C widened to fp32 into the root MMA's operand layout, and this tile's dt.
+#pragma unroll
+            for (int u = 0; u < kCItems; ++u) {
+                const int q = tid + u * kThreads, i = q >> 5, c = q & 31;
+                if (q < T_pad * 32) {
+                    float4 v;
+                    unpack4(craw[u], v.x, v.y, v.z, v.w);
+                    *reinterpret_cast<float4 *>(cs + (c >> 3) * T_pad * 128 + i * 128 + (((c & 7) ^ (i & 7)) << 4)) = v;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (tid + u * kThreads < hpt * T) coef(k & 1, 0)[tid + u * kThreads] = bf2f(dtv[u]);
             __syncthreads();
             // Phase 3: path rows of B (fp32) for the commit, C_i . B_j of every ancestor pair.
             if (misc[M_STATE] && p.tc_commit && misc[M_LEN] <= kPathRows) {
