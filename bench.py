@@ -55,7 +55,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample budget")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--layers", type=int, default=None, help="override the workload's layer count (profiling)")
-    ap.add_argument("--also", default="hyb8b,serve64,wide256,wide256_chain",
+    ap.add_argument("--also", default="tiny,hyb8b,serve64,wide256,wide256_chain",
                     help="comma-separated extra workloads summarised in the same line ('none' to skip)")
     ap.add_argument("--no-separate", action="store_true",
                     help="skip the stand-alone scan and commit timings")
