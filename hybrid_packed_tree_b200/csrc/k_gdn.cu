@@ -467,9 +467,18 @@ extern "C" stree_status stree_gdn_tree_scan_commit(const void *q, const void *k,
         return STREE_ERR_MISALIGNED;
     const long long grid = (long long)batch * heads_v * (dv / kRows);
     if (grid > 0x7fffffffLL) return STREE_ERR_UNSUPPORTED;
-    if (prepare_gdn() != cudaSuccess) return STREE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t *err = err_out;
+    if (gdn_tc_supported(n_nodes, dk, dv, dtype)) {
+        // The tensor-core kernel: one CTA per (sequence, value head).
+        if (err && cudaMemsetAsync(err, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return STREE_ERR_CUDA;
+        return launch_gdn_tc(q, k, v, alpha, beta, erase, S0, parent, n_nodes, batch, heads_v, heads_k,
+                             commit ? accepted_path : nullptr, commit ? path_len : nullptr, commit ? maxlen : 0, o,
+                             commit ? S_new : nullptr, err, s) == cudaSuccess
+                   ? STREE_OK
+                   : STREE_ERR_CUDA;
+    }
+    if (prepare_gdn() != cudaSuccess) return STREE_ERR_CUDA;
     if (err && cudaMemsetAsync(err, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return STREE_ERR_CUDA;
     GdnParams p{};
     p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.erase = erase; p.S0 = S0;

@@ -76,6 +76,13 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 // (0: every tree's pairs fit in its shared memory).
 size_t tc_pair_scratch_floats(const ScanArgs &a);
 
+// Gated delta rule on the tensor cores (bf16, d_k = d_v = 128, up to 64 nodes).
+bool gdn_tc_supported(int n_nodes, int dk, int dv, stree_dtype dtype);
+cudaError_t launch_gdn_tc(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+                          const float *erase, const float *S0, const int32_t *parent, int n_nodes, int batch,
+                          int heads_v, int heads_k, const int32_t *path, const int32_t *path_len, int maxlen, void *o,
+                          float *S_new, int32_t *err, cudaStream_t s);
+
 // Small-batch path: whether the shape is supported, and the launcher.
 bool small_supported(const ScanArgs &a);
 cudaError_t launch_scan_small(const ScanArgs &a, cudaStream_t s);

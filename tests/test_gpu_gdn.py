@@ -3,7 +3,8 @@ the fp64 oracle: every node's output and the committed state, element by element
 at the tolerances of the scan (1e-4 max|ref| for fp32 inputs, 2e-2 for bf16);
 invalid trees and paths, the empty path, the in-place commit and the call
 without a commit; the erase strength apart from the write strength (random, and
-zero: gated linear attention)."""
+zero: gated linear attention).  bf16 with d_v = 128 and up to 64 nodes runs the
+tensor-core kernel, every other shape the CUDA-core one; both are covered."""
 import numpy as np
 import pytest
 import torch
@@ -93,19 +94,24 @@ def test_gdn_decoupled_erase_matches_oracle(st, name, batch, hv, hk, dv, dtype, 
     assert_close(f64(S_new), S_ref, dtype, f"{name} S_new ({kind} erase)")
 
 
-def test_gdn_chain_of_64_and_empty_path_in_place(st):
+# (dv, dtype): the CUDA-core kernel, and the tensor-core kernel (bf16, d_v = 128).
+KERNEL_SHAPES = [(32, "f32"), (128, "bf16")]
+
+
+@pytest.mark.parametrize("dv,dtype", KERNEL_SHAPES)
+def test_gdn_chain_of_64_and_empty_path_in_place(st, dv, dtype):
     parent = np.stack([wl.chain_tree(64), wl.random_tree(np.random.default_rng(3), 64, max_depth=8)])
     path = np.full((2, 64), -1, np.int32)
     path[0, :40] = np.arange(40)
     plen = np.asarray([40, 0], np.int32)
-    g = wl.gdn_inputs(parent, path, plen, heads_v=2, heads_k=1, dv=32, dtype="f32", seed=5)
+    g = wl.gdn_inputs(parent, path, plen, heads_v=2, heads_k=1, dv=dv, dtype=dtype, seed=5)
     d = _upload(g)
     S0 = d["S0"].clone()
     o, _, err = _run(st, g, d, S_new=d["S0"])                        # commit in place over S0
     assert err == [0, 0, 0, 0]
     o_ref, S_ref = _oracle(g)
-    assert_close(f64(o), o_ref, "f32", "o")
-    assert_close(f64(d["S0"]), S_ref, "f32", "S_new in place")
+    assert_close(f64(o), o_ref, dtype, "o")
+    assert_close(f64(d["S0"]), S_ref, dtype, "S_new in place")
     assert torch.equal(d["S0"][1], S0[1])                            # empty path keeps S0 exactly
 
 
@@ -118,13 +124,14 @@ def test_gdn_without_commit(st):
     assert_close(f64(o), _oracle(g)[0], "bf16", "o")
 
 
-def test_gdn_bad_tree_and_bad_path(st):
+@pytest.mark.parametrize("dv,dtype", KERNEL_SHAPES)
+def test_gdn_bad_tree_and_bad_path(st, dv, dtype):
     par = [-1, 0, 0, 1, 1, 2]
     parent = np.asarray([par, par, par], np.int32)
     parent[1, 4] = 5                                                 # not topological
     path = np.asarray([[0, 1, 3, -1], [0, 1, -1, -1], [0, 2, 4, -1]], np.int32)   # 4 is not under 2
     plen = np.asarray([3, 2, 3], np.int32)
-    g = wl.gdn_inputs(parent, path, plen, heads_v=2, heads_k=1, dv=32, dtype="f32", seed=7)
+    g = wl.gdn_inputs(parent, path, plen, heads_v=2, heads_k=1, dv=dv, dtype=dtype, seed=7)
     d = _upload(g)
     o, S_new, err = _run(st, g, d)
     assert err[0] in (3, 4)
@@ -133,9 +140,9 @@ def test_gdn_bad_tree_and_bad_path(st):
     keep = [0]
     f = g.f64()
     o_ref = oracle_gdn_tree(*(f[k][keep] for k in ("q", "k", "v", "alpha", "beta", "S0")), parent[keep])
-    assert_close(f64(o[keep]), o_ref, "f32", "o of the valid sequence")
+    assert_close(f64(o[keep]), o_ref, dtype, "o of the valid sequence")
     S_ref = oracle_gdn_commit(*(f[k][keep] for k in ("k", "v", "alpha", "beta", "S0")), parent[keep], path[keep],
                               plen[keep])
-    assert_close(f64(S_new[keep]), S_ref, "f32", "S_new of the valid sequence")
+    assert_close(f64(S_new[keep]), S_ref, dtype, "S_new of the valid sequence")
     o_ref2 = oracle_gdn_tree(*(f[k][[2]] for k in ("q", "k", "v", "alpha", "beta", "S0")), parent[[2]])
-    assert_close(f64(o[[2]]), o_ref2, "f32", "o of the sequence with the bad path")
+    assert_close(f64(o[[2]]), o_ref2, dtype, "o of the sequence with the bad path")
