@@ -14,21 +14,21 @@
 // [128 x 128] fp32 (one TMA box, the 128-byte-swizzled K-major operand layout); q, k
 // and v arrive as bf16 TMA boxes beside it.  Every dense contraction of the rule
 // runs as one tf32 product on the tensor cores into tensor memory: R = S0 [Q;K]^T
-// (the root terms S0 q_i and S0 k_i of every node; M = 128 state rows, N = 128) and
+// (the root terms S0 q_i and S0 k_i of every node; M = 128 state rows, N = 128),
 // P = [Q;K] K^T (q_i . k_j and k_i . k_j of every node pair; M = 128, N = 64), q and
 // k widened to fp32 in the same operand layout (bf16 values are exact in tf32, so
-// only S0 is rounded, as in the SSM scan's root term).  The pair products, weighted
-// and masked to the ancestor relation, are stored transposed (row l holds node l's
-// weight in every later node) in the MN-major operand layout.  Then each of the 128
-// threads owns one state row and solves for its column of the pseudo-values in
-// blocks of up to 32 nodes held in registers, right-looking (node l's value is final
-// once the earlier nodes of its block are folded in, and is then folded into the
-// later ones with two-wide fp32 FMAs); the first block reaches the second through
-// one more tf32 product.  The outputs are a third product, U^T x (the q weights),
-// beside which the threads rebuild their rows of the accepted state in place over
-// the S0 tile, which one TMA store writes back.  Waits are bounded; a timeout
-// latches STREE_ERR_TIMEOUT and the CTA drains its copies and products before it
-// exits.
+// only S0 is rounded, as in the SSM scan's root term).  The pair products are
+// weighted and masked to the ancestor relation: the q weights as a K-major operand
+// (row i), the k weights as [l][j] (row l holds node l's weight in every later node)
+// for the solve.  Then each of the 128 threads owns one state row and solves for its
+// column of the pseudo-values in blocks of up to 32 nodes held in registers,
+// right-looking (node l's value is final once the earlier nodes of its block are
+// folded in, and is then folded into the later ones with two-wide fp32 FMAs); the
+// first block reaches the second through one more tf32 product.  The outputs are a
+// fourth product, U^T x (the q weights)^T, beside which the threads rebuild their
+// rows of the accepted state in place over the S0 tile; outputs and state leave by
+// TMA stores.  Waits are bounded; a timeout latches STREE_ERR_TIMEOUT and the CTA
+// drains its copies and products before it exits.
 #include <cuda.h>
 
 #include <climits>
