@@ -146,3 +146,26 @@ def test_gdn_bad_tree_and_bad_path(st, dv, dtype):
     assert_close(f64(S_new[keep]), S_ref, dtype, "S_new of the valid sequence")
     o_ref2 = oracle_gdn_tree(*(f[k][[2]] for k in ("q", "k", "v", "alpha", "beta", "S0")), parent[[2]])
     assert_close(f64(o[[2]]), o_ref2, dtype, "o of the sequence with the bad path")
+
+
+@pytest.mark.parametrize("T", [1, 2, 16, 17, 32, 33, 47, 63])
+def test_gdn_tensor_core_node_counts(st, T):
+    # The tensor-core kernel keeps 16, 32 or 64 nodes in registers and solves the
+    # second 32-node block after one product: node counts at and across those edges,
+    # a random tree and a chain, the random tree's path to its last node, the chain's
+    # whole length; a random erase strength for odd counts.
+    rng = np.random.default_rng(300 + T)
+    parent = np.stack([wl.random_tree(rng, T, max_depth=8), wl.chain_tree(T)]).astype(np.int32)
+    path = np.full((2, T), -1, np.int32)
+    p0 = wl.root_path_nodes(parent[0], T - 1)
+    path[0, :len(p0)] = p0
+    path[1, :T] = np.arange(T)
+    plen = np.asarray([len(p0), T], np.int32)
+    g = wl.gdn_inputs(parent, path, plen, heads_v=4, heads_k=2, dv=128, dtype="bf16", seed=50 + T)
+    er = np.random.default_rng(60 + T).uniform(0.0, 1.0, size=g.beta.shape).astype(np.float32) if T % 2 else None
+    d = _upload(g)
+    o, S_new, err = _run(st, g, d, erase=er)
+    assert err == [0, 0, 0, 0]
+    o_ref, S_ref = _oracle(g, erase=None if er is None else er.astype(np.float64))
+    assert_close(f64(o), o_ref, "bf16", f"T={T} o")
+    assert_close(f64(S_new), S_ref, "bf16", f"T={T} S_new")
