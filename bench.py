@@ -417,7 +417,9 @@ def run_gdn(name, local_rank, steps=50, heads_v=32, heads_k=16, linear=False):
     return {"workload": f"{name} trees, {rule} ({heads_v} value / {heads_k} key heads, d_k = d_v = 128)",
             "batch": b, "n_nodes": T, "ms_per_call": ms, "nodes_per_s": b * T / (ms / 1e3),
             "bytes_per_call": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs,
-            "peak_source": f"{peak_kind} hbm_gbs", "kernel": "gdn_tree_kernel",
+            "peak_source": f"{peak_kind} hbm_gbs",
+            # bf16, d = 128, up to 64 nodes: the tensor-core kernel; else the CUDA-core one
+            "kernel": "gdn_tc_kernel" if T <= 64 else "gdn_tree_kernel",
             "timing": f"{steps} calls in one CUDA graph after an L2 flush, {nsets} rotated buffer sets"}
 
 
