@@ -469,8 +469,10 @@ extern "C" stree_status stree_gdn_tree_scan_commit(const void *q, const void *k,
     if (grid > 0x7fffffffLL) return STREE_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t *err = err_out;
-    if (gdn_tc_supported(n_nodes, dk, dv, dtype)) {
-        // The tensor-core kernel: one CTA per (sequence, value head).
+    // The tensor-core kernel: one CTA per (sequence, value head); its state rows and
+    // node positions are 32-bit TMA coordinates.
+    if (gdn_tc_supported(n_nodes, dk, dv, dtype) && (long long)batch * heads_v * dv <= 0x7fffffffLL &&
+        (long long)batch * n_nodes <= 0x7fffffffLL) {
         if (err && cudaMemsetAsync(err, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return STREE_ERR_CUDA;
         return launch_gdn_tc(q, k, v, alpha, beta, erase, S0, parent, n_nodes, batch, heads_v, heads_k,
                              commit ? accepted_path : nullptr, commit ? path_len : nullptr, commit ? maxlen : 0, o,
