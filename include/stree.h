@@ -330,7 +330,9 @@ stree_status stree_accept_sampling(const void *target_logits, const void *draft_
  * accepted_path, path_len and S_new all NULL: no commit.
  *
  * Shapes: dk = 128, dv a multiple of 32 up to 256, n_nodes up to 64, heads_v a
- * multiple of heads_k (else STREE_ERR_UNSUPPORTED).  fp32 arithmetic throughout.
+ * multiple of heads_k (else STREE_ERR_UNSUPPORTED).  fp32 arithmetic; for bf16
+ * inputs with dv = 128 the contractions run on the tensor cores, which round S0,
+ * the pseudo-values and the pair weights to tf32 (fp32 accumulation).
  * An invalid tree latches STREE_ERR_BAD_TREE (that sequence's o and S_new are
  * untouched), an invalid path STREE_ERR_BAD_PATH (S_new untouched).  The caller
  * owns every buffer; the call allocates nothing and runs on `stream`.
